@@ -1,0 +1,92 @@
+"""Seeded synthetic inputs shared by the tests, the smoke check and the benchmark.
+
+This module draws random numbers and nothing else: it holds none of the
+W2A8 method's arithmetic (no ternarisation, no packing, no quantisation).
+Both the CPU oracle and the CUDA library receive the arrays it returns.
+
+Generator (counter based, so any element can be regenerated from its index):
+  * splitmix64 on the counter ``seed + (i + 1) * 0x9E3779B97F4A7C15``;
+  * 53-bit uniforms: u1 = ((z >> 11) + 1) * 2**-53 in (0, 1],
+    u2 = (z >> 11) * 2**-53 in [0, 1);
+  * Box-Muller in fp64 on the pair (2p, 2p+1): element 2p gets r*cos(theta),
+    element 2p+1 gets r*sin(theta); the result is rounded once to fp32.
+
+Seeds: ``seed_for(config, layer, matrix_id, kind)`` =
+``0xB17E7 ^ (config << 40) ^ (layer << 24) ^ (matrix_id << 16) ^ kind``.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+GOLDEN = np.uint64(0x9E3779B97F4A7C15)
+M1 = np.uint64(0xBF58476D1CE4E5B9)
+M2 = np.uint64(0x94D049BB133111EB)
+
+KIND_WEIGHT = 1
+KIND_ACT = 2
+KIND_OUTLIER = 3
+
+
+def seed_for(config: int, layer: int = 0, matrix_id: int = 0, kind: int = KIND_WEIGHT) -> int:
+    return (0xB17E7 ^ (config << 40) ^ (layer << 24) ^ (matrix_id << 16) ^ kind) & (2**64 - 1)
+
+
+def splitmix64(seed: int, counters: np.ndarray) -> np.ndarray:
+    """splitmix64 output for each counter value (uint64 array)."""
+    with np.errstate(over="ignore"):
+        z = np.uint64(seed) + (counters.astype(np.uint64) + np.uint64(1)) * GOLDEN
+        z = (z ^ (z >> np.uint64(30))) * M1
+        z = (z ^ (z >> np.uint64(27))) * M2
+        z = z ^ (z >> np.uint64(31))
+    return z
+
+
+def normal_f32(seed: int, n: int, start: int = 0) -> np.ndarray:
+    """Elements [start, start+n) of the seeded N(0,1) stream, as float32."""
+    if n <= 0:
+        return np.zeros(0, dtype=np.float32)
+    first_pair = start // 2
+    last_pair = (start + n - 1) // 2
+    pairs = np.arange(first_pair, last_pair + 1, dtype=np.uint64)
+    z1 = splitmix64(seed, 2 * pairs)
+    z2 = splitmix64(seed, 2 * pairs + np.uint64(1))
+    u1 = ((z1 >> np.uint64(11)).astype(np.float64) + 1.0) * 2.0**-53
+    u2 = (z2 >> np.uint64(11)).astype(np.float64) * 2.0**-53
+    r = np.sqrt(-2.0 * np.log(u1))
+    th = 2.0 * np.pi * u2
+    out = np.empty(2 * pairs.size, dtype=np.float64)
+    out[0::2] = r * np.cos(th)
+    out[1::2] = r * np.sin(th)
+    off = start - 2 * first_pair
+    return out[off:off + n].astype(np.float32)
+
+
+def normal_matrix(seed: int, rows: int, cols: int) -> np.ndarray:
+    return normal_f32(seed, rows * cols).reshape(rows, cols)
+
+
+def outlier_channels(seed: int, K: int, frac: float = 0.01) -> np.ndarray:
+    """floor(frac*K) channel indices, chosen by ranking splitmix64(seed, k)."""
+    n = int(np.floor(frac * K))
+    if n == 0:
+        return np.zeros(0, dtype=np.int64)
+    keys = splitmix64(seed, np.arange(K, dtype=np.uint64))
+    return np.sort(np.argsort(keys, kind="stable")[:n]).astype(np.int64)
+
+
+def activations(seed: int, T: int, K: int, outliers: bool = False, outlier_seed: int | None = None,
+                factor: float = 20.0) -> np.ndarray:
+    """fp32 N(0,1) activations [T][K]; optionally a fixed 1% of channels x factor."""
+    x = normal_matrix(seed, T, K)
+    if outliers:
+        ch = outlier_channels(outlier_seed if outlier_seed is not None else seed ^ KIND_OUTLIER, K)
+        x[:, ch] *= np.float32(factor)
+    return x
+
+
+def ternary_uniform(seed: int, rows: int, cols: int, p_zero: float = 0.31) -> np.ndarray:
+    """Random values in {-1, 0, +1} drawn directly (for layout and corner tests)."""
+    z = splitmix64(seed, np.arange(rows * cols, dtype=np.uint64))
+    u = (z >> np.uint64(11)).astype(np.float64) * 2.0**-53
+    t = np.where(u < p_zero, 0, np.where(u < p_zero + (1 - p_zero) / 2, -1, 1))
+    return t.astype(np.int8).reshape(rows, cols)
