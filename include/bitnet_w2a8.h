@@ -1,0 +1,210 @@
+/*
+ * bitnet_w2a8.h -- C ABI of libbitnet_w2a8.so, a B200 (sm_100a) library for
+ * the BitNet b1.58 ternary-weight x int8-activation ("W2A8") linear layer.
+ *
+ * What the layer computes, and where the pages say so:
+ *   - Weights are ternary {-1, 0, +1}, stored as "i2_s": 2-bit codes
+ *     0, 1, 2 for -1, 0, +1, four codes per byte, code shifted left by
+ *     (6 - 2*group_idx), 128-weight blocks with one float scale per block.
+ *     ("浏览器里跑 1-bit 大模型 BitNet WebAssembly 的 50 倍提速实操",
+ *     section "i2_s 到底是什么".)  group_idx is the index inside the block
+ *     divided by 32, so byte b of a block holds weights b, b+32, b+64, b+96.
+ *   - A packed row of `cols` weights takes cols/4 bytes ("BitRun v0.2
+ *     实测：1-bit LLM 终端驾驶舱与毫瓦级功耗遥测", section
+ *     "矩阵内存边界与步幅安全").
+ *   - Activations are 8-bit ("5倍性能跃升：BitNet与llama.cpp的1-bit LLM推理
+ *     架构对决", section "GPU内核突破"): per token, s = 127 / max(absmax,
+ *     1e-5) in fp32 and q = round-half-to-even(x * s), clamped to [-127, 127].
+ *   - The product is integer: +1 adds, -1 subtracts, 0 skips ("BitRun v0.2
+ *     实测", section "三值权重与 1.58-bit 的由来").  acc[b][o][j] is the int32
+ *     sum over block j, and y[b][o] = (sum_j scale[o][j] * acc[b][o][j]) / s[b]
+ *     ("i2_s 到底是什么": dequantisation is a lookup plus scaling).
+ *
+ * Conventions for every call:
+ *   - Row-major everywhere.  Weights are [rows = out][cols = K]; activations
+ *     are [T][K]; outputs are [T][out].  cols (K) must be a multiple of 128.
+ *   - The library never allocates and never frees caller memory.  Every
+ *     buffer is owned by the caller; device buffers may come from any CUDA
+ *     allocator (for example PyTorch).
+ *   - Device pointers named *_dev must be device memory on the current
+ *     device, 16-byte aligned unless a call says otherwise.
+ *   - Calls marked "async" validate their arguments on the host, enqueue
+ *     kernels on `stream` and return; errors found later on the device (a
+ *     bounded wait that ran out, a corrupt code) are latched in a per-device
+ *     error word read by bitnet_get_device_error().  Kernels never trap.
+ *   - A call that fails validation enqueues nothing and returns the status.
+ *     A launch failure returns BITNET_ERR_CUDA.
+ *   - bitnet_last_error_detail() gives a human-readable reason for the last
+ *     non-OK status returned on the calling host thread.
+ *   - NaN or Inf in activations or scales give unspecified (but memory-safe)
+ *     results.
+ */
+#ifndef BITNET_W2A8_H
+#define BITNET_W2A8_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; NULL selects the legacy default stream. */
+typedef struct CUstream_st *bitnet_stream_t;
+
+typedef enum {
+    BITNET_OK = 0,
+    BITNET_ERR_NULL = 1,        /* a required pointer is NULL               */
+    BITNET_ERR_SHAPE = 2,       /* a size is negative, too large, or K%128  */
+    BITNET_ERR_ALIGN = 3,       /* a pointer is not aligned as required     */
+    BITNET_ERR_VALUE = 4,       /* an input value is outside its domain     */
+    BITNET_ERR_CORRUPT = 5,     /* packed data holds the unused code 3      */
+    BITNET_ERR_BUFSIZE = 6,     /* a caller buffer is smaller than needed   */
+    BITNET_ERR_CUDA = 7,        /* a CUDA runtime call or launch failed     */
+    BITNET_ERR_TIMEOUT = 8,     /* a bounded device wait ran out            */
+    BITNET_ERR_UNSUPPORTED = 9  /* no kernel for this case / this device    */
+} bitnet_status;
+
+/* Static string naming a status.  Never NULL. */
+const char *bitnet_status_string(bitnet_status status);
+
+/* Reason for the last non-OK status on this host thread ("" if none). */
+const char *bitnet_last_error_detail(void);
+
+/* Library version, (major << 16) | minor. */
+uint32_t bitnet_version(void);
+
+/* ------------------------------------------------------------------------
+ * Sizes.  Return 0 for an invalid shape (negative, or cols % 128 != 0).
+ * ---------------------------------------------------------------------- */
+
+/* Bytes of i2_s codes for a rows x cols ternary matrix: rows * cols / 4. */
+size_t bitnet_i2s_code_bytes(int64_t rows, int64_t cols);
+
+/* Number of fp32 block scales: rows * cols / 128. */
+size_t bitnet_i2s_num_scales(int64_t rows, int64_t cols);
+
+/* Bytes of the device weight buffer that bitnet_repack_device fills. */
+size_t bitnet_repacked_bytes(int64_t rows, int64_t cols);
+
+/* ------------------------------------------------------------------------
+ * Host-side i2_s packing (plain, synchronous, no GPU needed).
+ * ---------------------------------------------------------------------- */
+
+/* Packs a row-major int8 matrix of {-1, 0, +1} into i2_s codes
+ * ("i2_s 到底是什么": -1 -> 0, 0 -> 1, +1 -> 2, code << (6 - 2*group_idx)).
+ * codes_out receives rows * cols / 4 bytes, row stride cols / 4.
+ * Errors: NULL, SHAPE, BUFSIZE (codes_bytes too small), VALUE (an entry is
+ * not in {-1, 0, +1}; codes_out is then unspecified). */
+bitnet_status bitnet_pack_i2s(const int8_t *ternary, int64_t rows, int64_t cols,
+                              uint8_t *codes_out, size_t codes_bytes);
+
+/* Inverse of bitnet_pack_i2s.  ternary_out receives rows * cols int8.
+ * Errors: NULL, SHAPE, BUFSIZE, CORRUPT (a 2-bit field holds code 3). */
+bitnet_status bitnet_unpack_i2s(const uint8_t *codes, int64_t rows, int64_t cols,
+                                int8_t *ternary_out, size_t ternary_bytes);
+
+/* ------------------------------------------------------------------------
+ * Device weights.
+ * ---------------------------------------------------------------------- */
+
+#define BITNET_LAYOUT_VERSION 1u
+/* flags filled in by bitnet_repack_device */
+#define BITNET_WEIGHT_UNIFORM_ROWS 1u /* every row's block scales are equal */
+
+typedef struct {
+    int64_t rows;            /* out */
+    int64_t cols;            /* K, multiple of 128 */
+    void *data;              /* device, caller-owned, 256-byte aligned     */
+    size_t bytes;            /* >= bitnet_repacked_bytes(rows, cols)       */
+    uint32_t layout_version; /* BITNET_LAYOUT_VERSION after a repack       */
+    uint32_t flags;          /* BITNET_WEIGHT_* after a repack             */
+} bitnet_weight;
+
+/* Converts i2_s codes [rows][cols/4] and block scales [rows][cols/128]
+ * (both device memory, left unchanged) into the kernels' device layout in
+ * w_out->data: 16-row x 128-column tiles of codes in the order the GEMV and
+ * GEMM kernels read them, the block scales per tile, and one scale per row
+ * when all of that row's block scales are equal.  The caller sets
+ * w_out->data and w_out->bytes; rows, cols, layout_version and flags are
+ * written here.  This call is once per weight and is SYNCHRONOUS: it waits
+ * for `stream` to read back the uniformity flag and the corruption check.
+ * codes_dev must be 4-byte aligned, scales_dev 4-byte aligned.
+ * Errors: NULL, SHAPE, ALIGN, BUFSIZE, CORRUPT (code 3 found; w_out is then
+ * unusable), CUDA. */
+bitnet_status bitnet_repack_device(const uint8_t *codes_dev, const float *scales_dev,
+                                   int64_t rows, int64_t cols, bitnet_weight *w_out,
+                                   bitnet_stream_t stream);
+
+/* Inverse of bitnet_repack_device (async): rewrites the i2_s codes
+ * [rows][cols/4] and block scales [rows][cols/128] from a repacked weight.
+ * Lets a caller check the device layout byte for byte. */
+bitnet_status bitnet_unrepack_device(const bitnet_weight *w, uint8_t *codes_out_dev,
+                                     float *scales_out_dev, bitnet_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Activation quantisation (async).
+ * ---------------------------------------------------------------------- */
+
+/* Per-row absmax int8 quantisation of fp32 x [T][K]:
+ *   s[t] = 127 / max(max_k |x[t][k]|, 1e-5)      (fp32, IEEE divide)
+ *   q[t][k] = clamp(rint(x[t][k] * s[t]), -127, 127)   (ties to even)
+ * q_dev receives T*K int8 (16-byte aligned), s_dev T fp32 (4-byte aligned).
+ * blocksum_dev (nullable, 4-byte aligned) receives T*(K/128) int32 sums of q
+ * over each 128-element block.  T may be 0 (nothing is launched).
+ * Errors: NULL, SHAPE, ALIGN, CUDA. */
+bitnet_status bitnet_quant_act(const float *x_dev, int64_t T, int64_t K, int8_t *q_dev,
+                               float *s_dev, int32_t *blocksum_dev, bitnet_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * The linear layer (async).
+ * ---------------------------------------------------------------------- */
+
+/* Decode / small-batch GEMV, 1 <= B <= 16:
+ *   y[b][o] = (sum_j scale[o][j] * acc[b][o][j]) / s[b]
+ * with acc the int32 block dot products of the ternary weights and q.
+ * q_dev: B*K int8 (16-byte aligned); s_dev: B fp32; y_dev: B*rows fp32
+ * (4-byte aligned).  The sum over blocks runs in fp64 and is rounded once.
+ * Errors: NULL, SHAPE (B outside 1..16, K mismatch), ALIGN, VALUE (w not
+ * repacked), CUDA. */
+bitnet_status bitnet_w2a8_gemv(const bitnet_weight *w, const int8_t *q_dev, const float *s_dev,
+                               int64_t B, float *y_dev, bitnet_stream_t stream);
+
+/* Prefill GEMM, T >= 1 tokens, same result as the GEMV (tcgen05 int8
+ * tensor cores, int32 accumulators in tensor memory).
+ * q_dev: T*K int8 (16-byte aligned); s_dev: T fp32; y_dev: T*rows fp32
+ * (16-byte aligned).  T = 0 launches nothing.
+ * Errors: NULL, SHAPE, ALIGN, VALUE, UNSUPPORTED (not an sm_100 device),
+ * CUDA.  Device-side bounded waits that run out latch BITNET_ERR_TIMEOUT. */
+bitnet_status bitnet_w2a8_gemm(const bitnet_weight *w, const int8_t *q_dev, const float *s_dev,
+                               int64_t T, float *y_dev, bitnet_stream_t stream);
+
+/* Test variants of the two calls above that also write the int32 block
+ * accumulators acc_dev[b][o][j], b < B (or T), o < rows, j < cols/128
+ * (4-byte aligned), so they can be compared bit for bit. */
+bitnet_status bitnet_w2a8_gemv_acc(const bitnet_weight *w, const int8_t *q_dev,
+                                   const float *s_dev, int64_t B, float *y_dev,
+                                   int32_t *acc_dev, bitnet_stream_t stream);
+bitnet_status bitnet_w2a8_gemm_acc(const bitnet_weight *w, const int8_t *q_dev,
+                                   const float *s_dev, int64_t T, float *y_dev,
+                                   int32_t *acc_dev, bitnet_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Device-side error reporting.
+ * ---------------------------------------------------------------------- */
+
+/* Waits for `stream`, then reads and clears the current device's error word:
+ * BITNET_OK, BITNET_ERR_TIMEOUT (a bounded wait ran out), BITNET_ERR_CORRUPT
+ * (a kernel met code 3) or BITNET_ERR_CUDA (the stream itself failed). */
+bitnet_status bitnet_get_device_error(bitnet_stream_t stream);
+
+/* Test hook: sets the iteration cap of the device-side bounded waits on the
+ * current device (0 restores the default).  A tiny cap makes a wait run out
+ * without hanging anything, so the timeout path can be exercised. */
+bitnet_status bitnet_set_wait_limit(uint32_t max_iterations);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BITNET_W2A8_H */

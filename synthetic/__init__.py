@@ -90,3 +90,20 @@ def ternary_uniform(seed: int, rows: int, cols: int, p_zero: float = 0.31) -> np
     u = (z >> np.uint64(11)).astype(np.float64) * 2.0**-53
     t = np.where(u < p_zero, 0, np.where(u < p_zero + (1 - p_zero) / 2, -1, 1))
     return t.astype(np.int8).reshape(rows, cols)
+
+
+def positive_scales(seed: int, rows: int, nb: int, uniform_per_row: bool = False,
+                    per_tensor: bool = False) -> np.ndarray:
+    """fp32 block scales [rows][nb] in [0.25, 4): 2**(4u - 2) for seeded uniforms u.
+
+    per_tensor: one value for the whole matrix; uniform_per_row: one value per row.
+    """
+    n = 1 if per_tensor else (rows if uniform_per_row else rows * nb)
+    z = splitmix64(seed, np.arange(n, dtype=np.uint64))
+    u = (z >> np.uint64(11)).astype(np.float64) * 2.0**-53
+    v = np.exp2(4.0 * u - 2.0).astype(np.float32)
+    if per_tensor:
+        return np.full((rows, nb), v[0], dtype=np.float32)
+    if uniform_per_row:
+        return np.repeat(v[:, None], nb, axis=1)
+    return v.reshape(rows, nb)

@@ -1,0 +1,320 @@
+// abi.cu -- the extern "C" entry points of libbitnet_w2a8.so: host-side
+// validation, dispatch to the kernels, status reporting, and the host i2_s
+// packer.  Declarations and their documentation: include/bitnet_w2a8.h.
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "common.cuh"
+
+namespace bitnet {
+
+__device__ unsigned g_error_word = 0u;
+__device__ unsigned g_wait_limit = kDefaultWaitLimit;
+
+namespace {
+
+thread_local char t_detail[256] = "";
+
+bitnet_status fail(bitnet_status st, const char *fmt, ...) __attribute__((format(printf, 2, 3)));
+bitnet_status fail(bitnet_status st, const char *fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(t_detail, sizeof(t_detail), fmt, ap);
+    va_end(ap);
+    return st;
+}
+
+bitnet_status cuda_fail(cudaError_t e, const char *what) {
+    return fail(BITNET_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned(const void *p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+constexpr int64_t kMaxCols = int64_t(1) << 20;
+constexpr int64_t kMaxRows = int64_t(1) << 31;
+constexpr int64_t kMaxT = int64_t(1) << 31;
+
+bool shape_ok(int64_t rows, int64_t cols) {
+    return rows >= 0 && cols >= 0 && cols % kQK == 0 && rows < kMaxRows && cols <= kMaxCols;
+}
+
+std::mutex g_mu;
+DeviceGlobals g_dev[64];
+bool g_dev_ok[64];
+
+bitnet_status check_weight(const bitnet_weight *w) {
+    if (!w) return fail(BITNET_ERR_NULL, "weight handle is NULL");
+    if (!w->data) return fail(BITNET_ERR_NULL, "weight data is NULL");
+    if (!shape_ok(w->rows, w->cols) || w->rows == 0 || w->cols == 0)
+        return fail(BITNET_ERR_SHAPE, "weight shape %lld x %lld invalid", (long long)w->rows,
+                    (long long)w->cols);
+    if (w->layout_version != BITNET_LAYOUT_VERSION)
+        return fail(BITNET_ERR_VALUE, "weight not repacked (layout_version %u)", w->layout_version);
+    if (!aligned(w->data, 256)) return fail(BITNET_ERR_ALIGN, "weight data not 256-byte aligned");
+    if (w->bytes < layout_of(w->rows, w->cols).total)
+        return fail(BITNET_ERR_BUFSIZE, "weight buffer %zu bytes, need %zu", w->bytes,
+                    layout_of(w->rows, w->cols).total);
+    return BITNET_OK;
+}
+
+}  // namespace
+
+cudaError_t device_globals(DeviceGlobals *out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_dev_ok[dev]) {
+        DeviceGlobals g;
+        e = cudaGetSymbolAddress((void **)&g.err, g_error_word);
+        if (e != cudaSuccess) return e;
+        e = cudaGetSymbolAddress((void **)&g.wait_limit, g_wait_limit);
+        if (e != cudaSuccess) return e;
+        g_dev[dev] = g;
+        g_dev_ok[dev] = true;
+    }
+    *out = g_dev[dev];
+    return cudaSuccess;
+}
+
+}  // namespace bitnet
+
+using namespace bitnet;
+
+extern "C" {
+
+const char *bitnet_status_string(bitnet_status s) {
+    switch (s) {
+        case BITNET_OK: return "BITNET_OK";
+        case BITNET_ERR_NULL: return "BITNET_ERR_NULL";
+        case BITNET_ERR_SHAPE: return "BITNET_ERR_SHAPE";
+        case BITNET_ERR_ALIGN: return "BITNET_ERR_ALIGN";
+        case BITNET_ERR_VALUE: return "BITNET_ERR_VALUE";
+        case BITNET_ERR_CORRUPT: return "BITNET_ERR_CORRUPT";
+        case BITNET_ERR_BUFSIZE: return "BITNET_ERR_BUFSIZE";
+        case BITNET_ERR_CUDA: return "BITNET_ERR_CUDA";
+        case BITNET_ERR_TIMEOUT: return "BITNET_ERR_TIMEOUT";
+        case BITNET_ERR_UNSUPPORTED: return "BITNET_ERR_UNSUPPORTED";
+    }
+    return "BITNET_ERR_UNKNOWN";
+}
+
+const char *bitnet_last_error_detail(void) { return t_detail; }
+
+uint32_t bitnet_version(void) { return (1u << 16) | 0u; }
+
+size_t bitnet_i2s_code_bytes(int64_t rows, int64_t cols) {
+    return shape_ok(rows, cols) ? (size_t)rows * (size_t)cols / 4 : 0;
+}
+
+size_t bitnet_i2s_num_scales(int64_t rows, int64_t cols) {
+    return shape_ok(rows, cols) ? (size_t)rows * (size_t)(cols / kQK) : 0;
+}
+
+size_t bitnet_repacked_bytes(int64_t rows, int64_t cols) {
+    return shape_ok(rows, cols) ? layout_of(rows, cols).total : 0;
+}
+
+// Host packer.  Byte (block*32 + i%32) of a row gets the code of weight i of
+// the block at shift 6 - 2*(i/32); the codes of a byte are gathered first so
+// every byte is written once.
+bitnet_status bitnet_pack_i2s(const int8_t *ternary, int64_t rows, int64_t cols,
+                              uint8_t *codes_out, size_t codes_bytes) {
+    t_detail[0] = 0;
+    if (!ternary || !codes_out) return fail(BITNET_ERR_NULL, "NULL pointer");
+    if (!shape_ok(rows, cols)) return fail(BITNET_ERR_SHAPE, "bad shape");
+    const size_t need = (size_t)rows * (size_t)cols / 4;
+    if (codes_bytes < need) return fail(BITNET_ERR_BUFSIZE, "codes buffer %zu < %zu", codes_bytes, need);
+    for (int64_t r = 0; r < rows; r++) {
+        const int8_t *src = ternary + r * cols;
+        uint8_t *dst = codes_out + r * (cols / 4);
+        for (int64_t blk = 0; blk < cols / kQK; blk++) {
+            const int8_t *w = src + blk * kQK;
+            for (int b = 0; b < 32; b++) {
+                unsigned byte = 0;
+                for (int grp = 0; grp < 4; grp++) {
+                    const int v = w[grp * 32 + b];
+                    if (v != -1 && v != 0 && v != 1)
+                        return fail(BITNET_ERR_VALUE, "value %d at row %lld col %lld is not ternary", v,
+                                    (long long)r, (long long)(blk * kQK + grp * 32 + b));
+                    byte |= (unsigned)(v + 1) << (6 - 2 * grp);
+                }
+                dst[blk * 32 + b] = (uint8_t)byte;
+            }
+        }
+    }
+    return BITNET_OK;
+}
+
+bitnet_status bitnet_unpack_i2s(const uint8_t *codes, int64_t rows, int64_t cols,
+                                int8_t *ternary_out, size_t ternary_bytes) {
+    t_detail[0] = 0;
+    if (!codes || !ternary_out) return fail(BITNET_ERR_NULL, "NULL pointer");
+    if (!shape_ok(rows, cols)) return fail(BITNET_ERR_SHAPE, "bad shape");
+    const size_t need = (size_t)rows * (size_t)cols;
+    if (ternary_bytes < need) return fail(BITNET_ERR_BUFSIZE, "output buffer %zu < %zu", ternary_bytes, need);
+    for (int64_t r = 0; r < rows; r++) {
+        const uint8_t *src = codes + r * (cols / 4);
+        int8_t *dst = ternary_out + r * cols;
+        for (int64_t blk = 0; blk < cols / kQK; blk++) {
+            for (int b = 0; b < 32; b++) {
+                const unsigned byte = src[blk * 32 + b];
+                for (int grp = 0; grp < 4; grp++) {
+                    const unsigned c = (byte >> (6 - 2 * grp)) & 3u;
+                    if (c == 3u)
+                        return fail(BITNET_ERR_CORRUPT, "code 3 at row %lld byte %lld", (long long)r,
+                                    (long long)(blk * 32 + b));
+                    dst[blk * kQK + grp * 32 + b] = (int8_t)((int)c - 1);
+                }
+            }
+        }
+    }
+    return BITNET_OK;
+}
+
+bitnet_status bitnet_repack_device(const uint8_t *codes_dev, const float *scales_dev, int64_t rows,
+                                   int64_t cols, bitnet_weight *w_out, bitnet_stream_t stream) {
+    t_detail[0] = 0;
+    if (!codes_dev || !scales_dev || !w_out || !w_out->data) return fail(BITNET_ERR_NULL, "NULL pointer");
+    if (!shape_ok(rows, cols) || rows == 0 || cols == 0)
+        return fail(BITNET_ERR_SHAPE, "shape %lld x %lld invalid", (long long)rows, (long long)cols);
+    if (!aligned(codes_dev, 4) || !aligned(scales_dev, 4) || !aligned(w_out->data, 256))
+        return fail(BITNET_ERR_ALIGN, "codes/scales need 4-byte, data 256-byte alignment");
+    const Layout L = layout_of(rows, cols);
+    if (w_out->bytes < L.total) return fail(BITNET_ERR_BUFSIZE, "data %zu < %zu bytes", w_out->bytes, L.total);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    w_out->layout_version = 0;
+    w_out->flags = 0;
+    cudaError_t e = launch_repack(codes_dev, scales_dev, rows, cols, w_out->data, st);
+    if (e != cudaSuccess) return cuda_fail(e, "repack launch");
+    unsigned hdr[2] = {0u, 0u};
+    e = cudaMemcpyAsync(hdr, w_out->data, sizeof(hdr), cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return cuda_fail(e, "repack readback");
+    if (hdr[1]) return fail(BITNET_ERR_CORRUPT, "packed codes hold code 3");
+    w_out->rows = rows;
+    w_out->cols = cols;
+    w_out->flags = hdr[0] == 0u ? BITNET_WEIGHT_UNIFORM_ROWS : 0u;
+    w_out->layout_version = BITNET_LAYOUT_VERSION;
+    return BITNET_OK;
+}
+
+bitnet_status bitnet_unrepack_device(const bitnet_weight *w, uint8_t *codes_out_dev,
+                                     float *scales_out_dev, bitnet_stream_t stream) {
+    t_detail[0] = 0;
+    bitnet_status s = check_weight(w);
+    if (s != BITNET_OK) return s;
+    if (!codes_out_dev || !scales_out_dev) return fail(BITNET_ERR_NULL, "NULL output");
+    if (!aligned(codes_out_dev, 4) || !aligned(scales_out_dev, 4))
+        return fail(BITNET_ERR_ALIGN, "outputs need 4-byte alignment");
+    cudaError_t e = launch_unrepack(w->data, w->rows, w->cols, codes_out_dev, scales_out_dev,
+                                    reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? BITNET_OK : cuda_fail(e, "unrepack launch");
+}
+
+bitnet_status bitnet_quant_act(const float *x_dev, int64_t T, int64_t K, int8_t *q_dev, float *s_dev,
+                               int32_t *blocksum_dev, bitnet_stream_t stream) {
+    t_detail[0] = 0;
+    if (T < 0 || T >= kMaxT || K <= 0 || K % kQK != 0 || K > kMaxCols)
+        return fail(BITNET_ERR_SHAPE, "T=%lld K=%lld invalid", (long long)T, (long long)K);
+    if (T == 0) return BITNET_OK;
+    if (!x_dev || !q_dev || !s_dev) return fail(BITNET_ERR_NULL, "NULL pointer");
+    if (!aligned(x_dev, 16) || !aligned(q_dev, 16) || !aligned(s_dev, 4) ||
+        (blocksum_dev && !aligned(blocksum_dev, 4)))
+        return fail(BITNET_ERR_ALIGN, "x and q need 16-byte, s and blocksum 4-byte alignment");
+    cudaError_t e = launch_quant_act(x_dev, T, K, q_dev, s_dev, blocksum_dev,
+                                     reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? BITNET_OK : cuda_fail(e, "quant_act launch");
+}
+
+static bitnet_status gemv_impl(const bitnet_weight *w, const int8_t *q_dev, const float *s_dev,
+                               int64_t B, float *y_dev, int32_t *acc_dev, bitnet_stream_t stream) {
+    t_detail[0] = 0;
+    bitnet_status s = check_weight(w);
+    if (s != BITNET_OK) return s;
+    if (B < 1 || B > 16) return fail(BITNET_ERR_SHAPE, "GEMV batch %lld outside 1..16", (long long)B);
+    if (!q_dev || !s_dev || !y_dev) return fail(BITNET_ERR_NULL, "NULL pointer");
+    if (!aligned(q_dev, 16) || !aligned(s_dev, 4) || !aligned(y_dev, 4) || (acc_dev && !aligned(acc_dev, 4)))
+        return fail(BITNET_ERR_ALIGN, "q needs 16-byte, s/y/acc 4-byte alignment");
+    cudaError_t e = launch_gemv(w->data, w->rows, w->cols, (w->flags & BITNET_WEIGHT_UNIFORM_ROWS) != 0,
+                                q_dev, s_dev, B, y_dev, acc_dev, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? BITNET_OK : cuda_fail(e, "gemv launch");
+}
+
+bitnet_status bitnet_w2a8_gemv(const bitnet_weight *w, const int8_t *q_dev, const float *s_dev, int64_t B,
+                               float *y_dev, bitnet_stream_t stream) {
+    return gemv_impl(w, q_dev, s_dev, B, y_dev, nullptr, stream);
+}
+
+bitnet_status bitnet_w2a8_gemv_acc(const bitnet_weight *w, const int8_t *q_dev, const float *s_dev,
+                                   int64_t B, float *y_dev, int32_t *acc_dev, bitnet_stream_t stream) {
+    if (!acc_dev) return fail(BITNET_ERR_NULL, "acc is NULL");
+    return gemv_impl(w, q_dev, s_dev, B, y_dev, acc_dev, stream);
+}
+
+static bitnet_status gemm_impl(const bitnet_weight *w, const int8_t *q_dev, const float *s_dev,
+                               int64_t T, float *y_dev, int32_t *acc_dev, bitnet_stream_t stream) {
+    t_detail[0] = 0;
+    bitnet_status s = check_weight(w);
+    if (s != BITNET_OK) return s;
+    if (T < 0 || T >= kMaxT) return fail(BITNET_ERR_SHAPE, "T=%lld invalid", (long long)T);
+    if (T == 0) return BITNET_OK;
+    if (!q_dev || !s_dev || !y_dev) return fail(BITNET_ERR_NULL, "NULL pointer");
+    if (!aligned(q_dev, 16) || !aligned(s_dev, 4) || !aligned(y_dev, 16) || (acc_dev && !aligned(acc_dev, 4)))
+        return fail(BITNET_ERR_ALIGN, "q and y need 16-byte, s/acc 4-byte alignment");
+    int dev = 0, major = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    if (e != cudaSuccess) return cuda_fail(e, "device query");
+    if (major != 10) return fail(BITNET_ERR_UNSUPPORTED, "GEMM needs an sm_100 device (found sm_%d)", major * 10);
+    DeviceGlobals g;
+    e = device_globals(&g);
+    if (e != cudaSuccess) return cuda_fail(e, "device globals");
+    e = launch_gemm(w->data, w->rows, w->cols, (w->flags & BITNET_WEIGHT_UNIFORM_ROWS) != 0, q_dev, s_dev,
+                    T, y_dev, acc_dev, g, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? BITNET_OK : cuda_fail(e, "gemm launch");
+}
+
+bitnet_status bitnet_w2a8_gemm(const bitnet_weight *w, const int8_t *q_dev, const float *s_dev, int64_t T,
+                               float *y_dev, bitnet_stream_t stream) {
+    return gemm_impl(w, q_dev, s_dev, T, y_dev, nullptr, stream);
+}
+
+bitnet_status bitnet_w2a8_gemm_acc(const bitnet_weight *w, const int8_t *q_dev, const float *s_dev,
+                                   int64_t T, float *y_dev, int32_t *acc_dev, bitnet_stream_t stream) {
+    if (!acc_dev) return fail(BITNET_ERR_NULL, "acc is NULL");
+    return gemm_impl(w, q_dev, s_dev, T, y_dev, acc_dev, stream);
+}
+
+bitnet_status bitnet_get_device_error(bitnet_stream_t stream) {
+    t_detail[0] = 0;
+    cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "stream");
+    DeviceGlobals g;
+    e = device_globals(&g);
+    if (e != cudaSuccess) return cuda_fail(e, "device globals");
+    unsigned word = 0;
+    e = cudaMemcpy(&word, g.err, sizeof(word), cudaMemcpyDeviceToHost);
+    if (e == cudaSuccess) e = cudaMemset(g.err, 0, sizeof(unsigned));
+    if (e != cudaSuccess) return cuda_fail(e, "error word");
+    if (word & kErrTimeout) return fail(BITNET_ERR_TIMEOUT, "a bounded device wait ran out (word 0x%x)", word);
+    if (word & kErrCorrupt) return fail(BITNET_ERR_CORRUPT, "a kernel met code 3 (word 0x%x)", word);
+    if (word) return fail(BITNET_ERR_VALUE, "device error word 0x%x", word);
+    return BITNET_OK;
+}
+
+bitnet_status bitnet_set_wait_limit(uint32_t max_iterations) {
+    t_detail[0] = 0;
+    DeviceGlobals g;
+    cudaError_t e = device_globals(&g);
+    if (e != cudaSuccess) return cuda_fail(e, "device globals");
+    const unsigned v = max_iterations ? max_iterations : kDefaultWaitLimit;
+    e = cudaMemcpy(g.wait_limit, &v, sizeof(v), cudaMemcpyHostToDevice);
+    return e == cudaSuccess ? BITNET_OK : cuda_fail(e, "wait limit");
+}
+
+}  // extern "C"

@@ -1,0 +1,76 @@
+// common.cuh -- internal declarations shared by the library's translation units.
+// Not part of the ABI (the ABI is include/bitnet_w2a8.h).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <stddef.h>
+
+#include "../../include/bitnet_w2a8.h"
+
+namespace bitnet {
+
+constexpr int kQK = 128;          // weights per i2_s block
+constexpr int kTileRows = 16;     // rows per device tile
+constexpr int kTileBytes = 512;   // 16 rows x 128 weights x 2 bits
+constexpr float kEps = 1e-5f;     // floor on absmax
+
+// Bits of the per-device error word.
+constexpr unsigned kErrTimeout = 1u;
+constexpr unsigned kErrCorrupt = 2u;
+constexpr unsigned kErrBounds = 4u;
+
+// Default iteration cap for bounded device waits.
+constexpr unsigned kDefaultWaitLimit = 1u << 26;
+
+static inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Byte layout of a repacked weight buffer (layout version 1).
+//   [0, 256)           header: u32 not_uniform_rows, u32 corrupt
+//   off_tiles          [ntr][nb][32 lanes][16 B] code tiles
+//   off_tscales        [ntr][nb][16] fp32 block scales, tile order
+//   off_rowscale       [ntr*16] fp32: the row's scale if all its block scales
+//                      are equal, else NaN
+struct Layout {
+    int64_t rows, cols, ntr, nb;
+    size_t off_tiles, off_tscales, off_rowscale, total;
+};
+
+static inline Layout layout_of(int64_t rows, int64_t cols) {
+    Layout L;
+    L.rows = rows;
+    L.cols = cols;
+    L.ntr = (rows + kTileRows - 1) / kTileRows;
+    L.nb = cols / kQK;
+    size_t tiles = (size_t)L.ntr * (size_t)L.nb * kTileBytes;
+    size_t tsc = (size_t)L.ntr * (size_t)L.nb * kTileRows * sizeof(float);
+    size_t rsc = (size_t)L.ntr * kTileRows * sizeof(float);
+    L.off_tiles = 256;
+    L.off_tscales = L.off_tiles + align_up(tiles, 256);
+    L.off_rowscale = L.off_tscales + align_up(tsc, 256);
+    L.total = L.off_rowscale + align_up(rsc, 256);
+    return L;
+}
+
+// Per-device addresses of the library's device globals.
+struct DeviceGlobals {
+    unsigned *err;         // error word (kErr* bits)
+    unsigned *wait_limit;  // iteration cap for bounded waits
+};
+cudaError_t device_globals(DeviceGlobals *out);
+
+// Launchers (return the launch error, if any).
+cudaError_t launch_quant_act(const float *x, int64_t T, int64_t K, int8_t *q, float *s,
+                             int32_t *blocksum, cudaStream_t st);
+cudaError_t launch_repack(const uint8_t *codes, const float *scales, int64_t rows, int64_t cols,
+                          void *data, cudaStream_t st);
+cudaError_t launch_unrepack(const void *data, int64_t rows, int64_t cols, uint8_t *codes,
+                            float *scales, cudaStream_t st);
+cudaError_t launch_gemv(const void *data, int64_t rows, int64_t cols, bool uniform,
+                        const int8_t *q, const float *s, int64_t B, float *y, int32_t *acc,
+                        cudaStream_t st);
+cudaError_t launch_gemm(const void *data, int64_t rows, int64_t cols, bool uniform,
+                        const int8_t *q, const float *s, int64_t T, float *y, int32_t *acc,
+                        const DeviceGlobals &g, cudaStream_t st);
+
+}  // namespace bitnet
