@@ -105,6 +105,33 @@ bitnet_status bitnet_unpack_i2s(const uint8_t *codes, int64_t rows, int64_t cols
                                 int8_t *ternary_out, size_t ternary_bytes);
 
 /* ------------------------------------------------------------------------
+ * Device-side absmean ternarisation + i2_s packing (async).
+ * ---------------------------------------------------------------------- */
+
+#define BITNET_ABSMEAN_PER_TENSOR 0 /* one gamma for the whole matrix       */
+#define BITNET_ABSMEAN_PER_BLOCK 1  /* one gamma per 128-weight block       */
+
+/* Bytes of device scratch bitnet_ternarize_absmean_device needs (any mode). */
+size_t bitnet_ternarize_workspace_bytes(int64_t rows, int64_t cols);
+
+/* Ternarises fp32 weights w_dev [rows][cols] with absmean scaling and packs
+ * them as i2_s ("浏览器里跑 1-bit 大模型 ..." sections "为什么是 WASM" and
+ * "i2_s 到底是什么"; "BitRun v0.2 实测" section "三值权重与 1.58-bit 的由来"):
+ *   gamma = max(mean |W| (fp64 sum, rounded once to fp32), 1e-5)
+ *   t = clamp(rint(W / gamma), -1, 1)  (fp32 divide, ties to even)
+ * over the whole matrix (PER_TENSOR) or over each 128-weight block
+ * (PER_BLOCK).  Writes codes_out_dev [rows][cols/4] (4-byte aligned) and the
+ * block scales scales_out_dev [rows][cols/128] (every one equal to gamma in
+ * PER_TENSOR mode).  workspace_dev (>= bitnet_ternarize_workspace_bytes,
+ * 16-byte aligned, contents ignored) is caller-owned scratch; the per-tensor
+ * reduction runs in a fixed order, so results are reproducible bit for bit.
+ * Errors: NULL, SHAPE, ALIGN, BUFSIZE, VALUE (unknown mode), CUDA. */
+bitnet_status bitnet_ternarize_absmean_device(const float *w_dev, int64_t rows, int64_t cols, int mode,
+                                              uint8_t *codes_out_dev, float *scales_out_dev,
+                                              void *workspace_dev, size_t workspace_bytes,
+                                              bitnet_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * Device weights.
  * ---------------------------------------------------------------------- */
 

@@ -32,6 +32,8 @@ BITNET_ERR_CUDA = 7
 BITNET_ERR_TIMEOUT = 8
 BITNET_ERR_UNSUPPORTED = 9
 
+BITNET_ABSMEAN_PER_TENSOR = 0
+BITNET_ABSMEAN_PER_BLOCK = 1
 BITNET_LAYOUT_VERSION = 1
 BITNET_WEIGHT_UNIFORM_ROWS = 1
 QK = 128
@@ -66,6 +68,8 @@ def _load() -> ctypes.CDLL:
         "bitnet_repacked_bytes": ([i64, i64], sz),
         "bitnet_pack_i2s": ([vp, i64, i64, vp, sz], st),
         "bitnet_unpack_i2s": ([vp, i64, i64, vp, sz], st),
+        "bitnet_ternarize_workspace_bytes": ([i64, i64], sz),
+        "bitnet_ternarize_absmean_device": ([vp, i64, i64, ctypes.c_int, vp, vp, vp, sz, vp], st),
         "bitnet_repack_device": ([vp, vp, i64, i64, W, vp], st),
         "bitnet_unrepack_device": ([W, vp, vp, vp], st),
         "bitnet_quant_act": ([vp, i64, i64, vp, vp, vp, vp], st),
@@ -166,6 +170,21 @@ def bitnet_unpack_i2s(codes: np.ndarray, cols: int) -> np.ndarray:
 
 
 # ---------------------------------------------------------------- device --
+
+def bitnet_ternarize_workspace_bytes(rows: int, cols: int) -> int:
+    return _lib.bitnet_ternarize_workspace_bytes(rows, cols)
+
+
+def bitnet_ternarize_absmean_device(w, rows: int, cols: int, mode: int, codes_out, scales_out, workspace,
+                                    stream=None):
+    """fp32 w [rows*cols] -> i2_s codes uint8 [rows*cols/4] and fp32 block scales (CUDA tensors)."""
+    _check(_lib.bitnet_ternarize_absmean_device(
+        _dptr(w, "float32", rows * cols, "w"), rows, cols, mode,
+        _dptr(codes_out, "uint8", rows * cols // 4, "codes"),
+        _dptr(scales_out, "float32", rows * cols // QK, "scales"),
+        _dptr(workspace, "uint8", bitnet_ternarize_workspace_bytes(rows, cols), "workspace"),
+        workspace.numel(), _stream(stream)), "bitnet_ternarize_absmean_device")
+
 
 class Weight:
     """A repacked device weight: the C struct plus the buffer that backs it."""

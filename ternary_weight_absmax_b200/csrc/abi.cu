@@ -176,6 +176,35 @@ bitnet_status bitnet_unpack_i2s(const uint8_t *codes, int64_t rows, int64_t cols
     return BITNET_OK;
 }
 
+size_t bitnet_ternarize_workspace_bytes(int64_t rows, int64_t cols) {
+    if (!shape_ok(rows, cols)) return 0;
+    return (size_t)absmean_num_partials(rows * cols) * sizeof(double) + 256;
+}
+
+bitnet_status bitnet_ternarize_absmean_device(const float *w_dev, int64_t rows, int64_t cols, int mode,
+                                              uint8_t *codes_out_dev, float *scales_out_dev,
+                                              void *workspace_dev, size_t workspace_bytes,
+                                              bitnet_stream_t stream) {
+    t_detail[0] = 0;
+    if (!shape_ok(rows, cols)) return fail(BITNET_ERR_SHAPE, "shape %lld x %lld invalid", (long long)rows,
+                                           (long long)cols);
+    if (mode != BITNET_ABSMEAN_PER_TENSOR && mode != BITNET_ABSMEAN_PER_BLOCK)
+        return fail(BITNET_ERR_VALUE, "unknown mode %d", mode);
+    if (rows == 0 || cols == 0) return BITNET_OK;
+    if (!w_dev || !codes_out_dev || !scales_out_dev || !workspace_dev) return fail(BITNET_ERR_NULL, "NULL pointer");
+    if (!aligned(w_dev, 4) || !aligned(codes_out_dev, 4) || !aligned(scales_out_dev, 4) ||
+        !aligned(workspace_dev, 16))
+        return fail(BITNET_ERR_ALIGN, "w/codes/scales need 4-byte, workspace 16-byte alignment");
+    const size_t need = bitnet_ternarize_workspace_bytes(rows, cols);
+    if (workspace_bytes < need) return fail(BITNET_ERR_BUFSIZE, "workspace %zu < %zu bytes", workspace_bytes, need);
+    double *partials = static_cast<double *>(workspace_dev);
+    float *gamma_slot = reinterpret_cast<float *>(static_cast<char *>(workspace_dev) + need - 256);
+    cudaError_t e = launch_ternarize(w_dev, rows, cols, mode == BITNET_ABSMEAN_PER_BLOCK,
+                                     reinterpret_cast<uint32_t *>(codes_out_dev), scales_out_dev, partials,
+                                     gamma_slot, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? BITNET_OK : cuda_fail(e, "ternarize launch");
+}
+
 bitnet_status bitnet_repack_device(const uint8_t *codes_dev, const float *scales_dev, int64_t rows,
                                    int64_t cols, bitnet_weight *w_out, bitnet_stream_t stream) {
     t_detail[0] = 0;

@@ -69,6 +69,9 @@ cudaError_t launch_unrepack(const void *data, int64_t rows, int64_t cols, uint8_
 cudaError_t launch_gemv(const void *data, int64_t rows, int64_t cols, bool uniform,
                         const int8_t *q, const float *s, int64_t B, float *y, int32_t *acc,
                         cudaStream_t st);
+int absmean_num_partials(int64_t n);
+cudaError_t launch_ternarize(const float *w, int64_t rows, int64_t cols, bool per_block, uint32_t *codes,
+                             float *scales, double *partials, float *gamma_slot, cudaStream_t st);
 cudaError_t launch_gemm(const void *data, int64_t rows, int64_t cols, bool uniform,
                         const int8_t *q, const float *s, int64_t T, float *y, int32_t *acc,
                         const DeviceGlobals &g, cudaStream_t st);

@@ -210,3 +210,139 @@ def test_gemv_full_size_sampled_rows(rows, K, B):
     pick = pick.astype(np.int64)
     ref = oracle.linear(oracle.pack_i2s(t[pick]), sc[pick], K, rq, rs)
     np.testing.assert_array_equal(y[:, pick], ref)
+
+
+# ------------------------------------------------------ device ternarise --
+
+def _gpu_ternarize(w, mode):
+    b = lib()
+    tt = torch()
+    rows, cols = w.shape
+    codes = tt.empty(rows * cols // 4, dtype=tt.uint8, device="cuda")
+    scales = tt.empty(rows * cols // QK, dtype=tt.float32, device="cuda")
+    ws = tt.full((b.bitnet_ternarize_workspace_bytes(rows, cols),), 0xAB, dtype=tt.uint8, device="cuda")
+    b.bitnet_ternarize_absmean_device(cuda(w.reshape(-1)), rows, cols, mode, codes, scales, ws)
+    return to_np(codes).reshape(rows, cols // 4), to_np(scales).reshape(rows, cols // QK)
+
+
+@pytest.mark.parametrize("rows,cols", [(1, 128), (256, 512), (1000, 640), (3840, 2560), (2560, 6912)])
+def test_ternarize_per_block_bit_exact(rows, cols):
+    w = syn.normal_matrix(syn.seed_for(2, 0, rows % 251, syn.KIND_WEIGHT), rows, cols)
+    w[0, :128] = 0.0                                             # all-zero block -> 1e-5 floor
+    codes, scales = _gpu_ternarize(w, lib().BITNET_ABSMEAN_PER_BLOCK)
+    t, sc = oracle.absmean_blocks(w)
+    np.testing.assert_array_equal(scales, sc)
+    np.testing.assert_array_equal(codes, oracle.pack_i2s(t))
+
+
+@pytest.mark.parametrize("rows,cols", [(256, 512), (3840, 2560), (13824, 2560), (4096, 14336)])
+def test_ternarize_per_tensor(rows, cols):
+    # gamma is an fp64 sum rounded to fp32; the library adds in a fixed tree
+    # order and the oracle left to right, so the two gammas may differ by one
+    # fp32 ulp in rare cases.  Then, and only then, codes may differ, and only
+    # where |W/gamma| sits at a rounding boundary.
+    w = syn.normal_matrix(syn.seed_for(3, 0, rows % 251, syn.KIND_WEIGHT), rows, cols)
+    codes, scales = _gpu_ternarize(w, lib().BITNET_ABSMEAN_PER_TENSOR)
+    t, g = oracle.absmean_tensor(w)
+    assert np.all(scales == scales.flat[0])
+    g_gpu = scales.flat[0]
+    assert abs(int(g_gpu.view(np.int32)) - int(np.float32(g).view(np.int32))) <= 1
+    if g_gpu == g:
+        np.testing.assert_array_equal(codes, oracle.pack_i2s(t))
+    else:
+        t_gpu = oracle.unpack_i2s(codes, cols)
+        diff = t_gpu != t
+        r = np.abs(w[diff] / np.float32(g))
+        assert np.all(np.abs(r - np.round(r - 0.5) - 0.5) < 1e-6)
+
+
+def test_ternarize_zero_fraction():
+    rows, cols = 4096, 4096
+    w = syn.normal_matrix(17, rows, cols)
+    codes, _ = _gpu_ternarize(w, lib().BITNET_ABSMEAN_PER_TENSOR)
+    frac = float(np.mean(oracle.unpack_i2s(codes, cols) == 0))
+    assert 0.305 <= frac <= 0.315
+
+
+# ------------------------------------------------------------------ GEMM --
+
+def _run_gemm(t, sc, x, with_acc=False, guard=64):
+    b = lib()
+    tt = torch()
+    rows, K = t.shape
+    T = x.shape[0]
+    w, _ = device_weight(t, sc)
+    q, s, _ = gpu_quant(x)
+    ybuf = tt.full((T * rows + 2 * guard,), 12345.0, dtype=tt.float32, device="cuda")
+    y = ybuf[guard:guard + T * rows]
+    acc = None
+    if with_acc:
+        acc = tt.full((T * rows * (K // QK),), -7, dtype=tt.int32, device="cuda")
+        b.bitnet_w2a8_gemm_acc(w, q, s, T, y, acc)
+    else:
+        b.bitnet_w2a8_gemm(w, q, s, T, y)
+    assert b.bitnet_get_device_error() == b.BITNET_OK
+    yb = to_np(ybuf)
+    assert np.all(yb[:guard] == 12345.0) and np.all(yb[guard + T * rows:] == 12345.0), "output guard overwritten"
+    return w, to_np(q).reshape(T, K), to_np(s), to_np(y).reshape(T, rows), \
+        (to_np(acc).reshape(T, rows, K // QK) if acc is not None else None)
+
+
+@pytest.mark.parametrize("rows,K,T,mode", [
+    (256, 512, 40, "tensor"), (256, 512, 40, "block"),
+    (1, 128, 1, "tensor"), (17, 128, 33, "block"), (100, 384, 129, "tensor"), (1000, 640, 200, "row"),
+    (300, 256, 512, "tensor"), (2560, 2560, 256, "tensor"), (2560, 2560, 256, "block"),
+])
+def test_gemm_matches_oracle(rows, K, T, mode):
+    t, sc, x = _gemv_case(rows, K, T, mode, seed=rows * 17 + K + T)
+    _, q, s, y, _ = _run_gemm(t, sc, x)
+    rq, rs, _ = oracle.quant_act(x)
+    np.testing.assert_array_equal(q, rq)
+    ref = oracle.linear(oracle.pack_i2s(t), sc, K, rq, rs)
+    assert_close(y, ref, f"gemm {rows}x{K} T={T} {mode}")
+
+
+@pytest.mark.parametrize("rows,K,T", [(64, 256, 1), (200, 384, 130), (513, 1280, 77)])
+def test_gemm_block_accumulators_bit_exact(rows, K, T):
+    t, sc, x = _gemv_case(rows, K, T, "block", seed=rows + 5 * K + T)
+    _, q, s, y, acc = _run_gemm(t, sc, x, with_acc=True)
+    rq, rs, _ = oracle.quant_act(x)
+    np.testing.assert_array_equal(acc, oracle.block_acc(oracle.pack_i2s(t), K, rq))
+    assert_close(y, oracle.linear(oracle.pack_i2s(t), sc, K, rq, rs), "gemm_acc y")
+
+
+def test_gemm_agrees_with_gemv_on_small_batches():
+    rows, K = 2560, 2560
+    for T in (1, 5, 16):
+        t, sc, x = _gemv_case(rows, K, T, "tensor", seed=31 + T)
+        _, _, _, _, yg, _ = _run_gemv(t, sc, x)
+        _, _, _, ym, _ = _run_gemm(t, sc, x)
+        assert_close(ym, yg, f"gemm vs gemv T={T}")
+
+
+@pytest.mark.parametrize("rows,K,T", [(13824, 2560, 512), (2560, 6912, 512), (13824, 2560, 2048),
+                                      (2560, 6912, 2048), (28672, 4096, 1024), (4096, 14336, 1024)])
+def test_gemm_full_size_sampled(rows, K, T):
+    # Full-size prefill as the benchmark launches it; the oracle checks a
+    # seeded sample of output rows for every token.
+    t, sc, x = _gemv_case(rows, K, T, "tensor", seed=rows ^ K ^ T, outliers=True)
+    _, q, s, y, _ = _run_gemm(t, sc, x)
+    rq, rs, _ = oracle.quant_act(x)
+    np.testing.assert_array_equal(q, rq)
+    pick = np.unique(np.concatenate([[0, rows - 1], syn.splitmix64(rows + T, np.arange(30)) % np.uint64(rows)]))
+    pick = pick.astype(np.int64)
+    ref = oracle.linear(oracle.pack_i2s(t[pick]), sc[pick], K, rq, rs)
+    assert_close(y[:, pick], ref, f"gemm full {rows}x{K} T={T}")
+
+
+def test_gemm_zero_tokens_is_a_no_op():
+    b = lib()
+    tt = torch()
+    t, sc, x = _gemv_case(64, 256, 1, "tensor", seed=3)
+    w, _ = device_weight(t, sc)
+    y = tt.full((64,), 5.0, device="cuda")
+    q = tt.zeros(256, dtype=tt.int8, device="cuda")
+    s = tt.ones(1, device="cuda")
+    b.bitnet_w2a8_gemm(w, q, s, 0, y)
+    assert b.bitnet_get_device_error() == b.BITNET_OK
+    assert np.all(to_np(y) == 5.0)
