@@ -131,6 +131,28 @@ bitnet_status bitnet_ternarize_absmean_device(const float *w_dev, int64_t rows, 
                                               void *workspace_dev, size_t workspace_bytes,
                                               bitnet_stream_t stream);
 
+/* Same as bitnet_ternarize_absmean_device, for callers that cannot allocate
+ * device memory: no workspace argument.  The pages have no counterpart; this
+ * entry point exists because some callers cannot hand the library scratch
+ * memory -- a host whose own fixed pool already owns all device memory, a
+ * binding with no device allocator, or a serving loop that must not call
+ * cudaMalloc (it may synchronise the device).  The scratch instead lives in a
+ * static device array inside the library, 2048 * 8 + 256 = 16640 bytes, which
+ * every GPU that loads the library keeps until the process exits; a request
+ * needing more (none with today's fixed reduction grid) is refused with
+ * BITNET_ERR_BUFSIZE.  The array is shared by all calls on a device and keeps
+ * the last call's contents (nothing in it has to start at zero): calls that
+ * overlap on the GPU -- on different streams, or from different host
+ * threads -- race on it and must be serialised by the caller.  The first call
+ * on each device looks the array's address up (cudaGetSymbolAddress, with
+ * that device current) and caches it; make that first call before any stream
+ * capture.  Calls no cudaMalloc, cudaFree or allocating library routine.
+ * Errors: as bitnet_ternarize_absmean_device, plus BUFSIZE as above and CUDA
+ * if the address lookup fails. */
+bitnet_status bitnet_ternarize_absmean_device_noalloc(const float *w_dev, int64_t rows, int64_t cols, int mode,
+                                                      uint8_t *codes_out_dev, float *scales_out_dev,
+                                                      bitnet_stream_t stream);
+
 /* ------------------------------------------------------------------------
  * Device weights.
  * ---------------------------------------------------------------------- */

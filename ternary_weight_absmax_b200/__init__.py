@@ -70,6 +70,7 @@ def _load() -> ctypes.CDLL:
         "bitnet_unpack_i2s": ([vp, i64, i64, vp, sz], st),
         "bitnet_ternarize_workspace_bytes": ([i64, i64], sz),
         "bitnet_ternarize_absmean_device": ([vp, i64, i64, ctypes.c_int, vp, vp, vp, sz, vp], st),
+        "bitnet_ternarize_absmean_device_noalloc": ([vp, i64, i64, ctypes.c_int, vp, vp, vp], st),
         "bitnet_repack_device": ([vp, vp, i64, i64, W, vp], st),
         "bitnet_unrepack_device": ([W, vp, vp, vp], st),
         "bitnet_quant_act": ([vp, i64, i64, vp, vp, vp, vp], st),
@@ -207,6 +208,17 @@ class Weight:
 
     def ref(self):
         return ctypes.byref(self.struct)
+
+
+def bitnet_ternarize_absmean_device_noalloc(w, rows: int, cols: int, mode: int, codes_out, scales_out,
+                                            stream=None):
+    """As bitnet_ternarize_absmean_device, with the library's static scratch
+    instead of a caller workspace (for callers that cannot allocate)."""
+    _check(_lib.bitnet_ternarize_absmean_device_noalloc(
+        _dptr(w, "float32", rows * cols, "w"), rows, cols, mode,
+        _dptr(codes_out, "uint8", rows * cols // 4, "codes"),
+        _dptr(scales_out, "float32", rows * cols // QK, "scales"), _stream(stream)),
+        "bitnet_ternarize_absmean_device_noalloc")
 
 
 def bitnet_repack_device(codes_dev, scales_dev, rows: int, cols: int, data_dev, stream=None) -> Weight:

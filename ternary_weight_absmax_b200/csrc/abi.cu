@@ -62,6 +62,14 @@ bitnet_status check_weight(const bitnet_weight *w) {
 
 }  // namespace
 
+bitnet_status set_error_detail(bitnet_status st, const char *fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(t_detail, sizeof(t_detail), fmt, ap);
+    va_end(ap);
+    return st;
+}
+
 cudaError_t device_globals(DeviceGlobals *out) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);

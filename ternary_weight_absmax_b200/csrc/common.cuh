@@ -52,6 +52,10 @@ static inline Layout layout_of(int64_t rows, int64_t cols) {
     return L;
 }
 
+// Records a human-readable reason for `st` (returned by
+// bitnet_last_error_detail on this host thread) and returns `st`.
+bitnet_status set_error_detail(bitnet_status st, const char *fmt, ...) __attribute__((format(printf, 2, 3)));
+
 // Per-device addresses of the library's device globals.
 struct DeviceGlobals {
     unsigned *err;         // error word (kErr* bits)
