@@ -3,15 +3,17 @@
 Default workload (one step): the decode linears of a BitNet-b1.58-2B-shaped
 model at batch 1 -- 30 layers x {QKV 3840x2560, O 2560x2560, gate+up
 13824x2560, down 2560x6912}, each with its own seeded weights and input.
-Per linear: bitnet_quant_act (fp32 x -> int8 q, s) then bitnet_w2a8_gemv.
-The 240 C-ABI calls of a step are captured once in a CUDA graph and the graph
-is replayed; the 520 MB of packed weights exceed the 126 MB L2, so every step
-streams them from HBM.
+Per linear: bitnet_w2a8_linear (fp32 x -> int8 q, s -> GEMV -> fp32 y, one
+kernel).  The 120 C-ABI calls of a step are captured once in a CUDA graph and
+the graph is replayed; the 520 MB of packed weights exceed the 126 MB L2, so
+every step streams them from HBM.  The two-call path (bitnet_quant_act then
+bitnet_w2a8_gemv) is timed the same way and reported beside it.
 
 Metric: achieved HBM GB/s = algorithmic bytes of a step / device time (higher
 is better).  Algorithmic bytes per linear: packed codes out*K/4 + one fp32
-scale per row (uniform per-tensor absmean scale) + q (K) + s (4) + y (4*out)
-for the GEMV, and x (4K) + q (K) + s (4) for the quantiser.
+scale per row (uniform per-tensor absmean scale) + x (4K) + y (4*out); the
+two-call path adds the q (K) and s (4) round trip and the GEMV alone counts
+codes + row scales + q + s + y.
 
 Also reported in the same JSON line: per-shape GEMV microseconds and GB/s
 (L2 flushed before each timed pass), the prefill GEMM int8 TOPS
@@ -56,6 +58,15 @@ def step_bytes(shapes=SHAPES, layers=LAYERS, B=1):
 
 def gemv_bytes(out, K, B=1):
     return out * K // 4 + 4 * out + B * K + 4 * B + 4 * B * out
+
+
+def linear_bytes(out, K, B=1):
+    """Fused path: packed codes + row scales + fp32 x in + fp32 y out."""
+    return out * K // 4 + 4 * out + 4 * B * K + 4 * B * out
+
+
+def fused_step_bytes(shapes=SHAPES, layers=LAYERS, B=1):
+    return sum(linear_bytes(o, k, B) for _, o, k in shapes) * layers
 
 
 def reduce_max(values, device):
@@ -214,6 +225,7 @@ def run_ours(args, rank, world, dev):
     launches_per_step = 0
 
     def step(gemv_only=False, only=None):
+        """Two C-ABI calls per linear: bitnet_quant_act, bitnet_w2a8_gemv."""
         n = 0
         for l in range(LAYERS):
             for name, o, k in SHAPES:
@@ -228,6 +240,17 @@ def run_ours(args, rank, world, dev):
                 n += 1
         return n
 
+    def fused_step():
+        """One C-ABI call per linear: bitnet_w2a8_linear (quantise + GEMV)."""
+        n = 0
+        for l in range(LAYERS):
+            for name, o, k in SHAPES:
+                key = (l, name)
+                xo, xn = xviews[key]
+                b.bitnet_w2a8_linear(weights[key], x_dev[xo:xo + xn], B, yviews[key])
+                n += 1
+        return n
+
     # Warm the quantised inputs once so GEMV-only graphs read real q, s.
     with torch.cuda.stream(stream):
         step()
@@ -239,7 +262,8 @@ def run_ours(args, rank, world, dev):
             cnt = fn()
         return g, cnt
 
-    g_step, launches_per_step = capture(lambda: step())
+    g_step, launches_per_step = capture(fused_step)
+    g_two, two_launches = capture(lambda: step())
     g_gemv, gemv_launches = capture(lambda: step(gemv_only=True))
     g_shape = {name: capture(lambda name=name: step(gemv_only=True, only=name))[0] for name, _, _ in SHAPES}
     flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
@@ -286,6 +310,9 @@ def run_ours(args, rank, world, dev):
     step_ms_local = e0.elapsed_time(e1) / args.steps
     clocks.stop()
 
+    # ---- the two-call path (bitnet_quant_act + bitnet_w2a8_gemv) ----
+    two_ms = timed(g_two, max(3, min(50, args.steps)))
+    two_ms_step = sorted(two_ms)[len(two_ms) // 2]
     # ---- GEMV-only replays (roofline of the dominant kernel) ----
     gemv_ms = timed(g_gemv, max(3, min(20, args.steps)))
     gemv_ms_per_step = sorted(gemv_ms)[len(gemv_ms) // 2]
@@ -326,8 +353,9 @@ def run_ours(args, rank, world, dev):
         raise RuntimeError(f"device error after bench: {b.bitnet_status_string(status)}")
 
     gbytes, qbytes = step_bytes()
-    per_rank_bytes = gbytes + qbytes
-    step_ms, e2e_ms, gemv_ms_max = reduce_max([step_ms_local, e2e_ms_local, gemv_ms_per_step], dev)
+    per_rank_bytes = fused_step_bytes()
+    step_ms, e2e_ms, gemv_ms_max, two_ms_max = reduce_max(
+        [step_ms_local, e2e_ms_local, gemv_ms_per_step, two_ms_step], dev)
     value, _ = aggregate([step_ms] * world, [per_rank_bytes] * world)
     e2e_value, _ = aggregate([e2e_ms] * world, [per_rank_bytes] * world)
 
@@ -346,12 +374,17 @@ def run_ours(args, rank, world, dev):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_ms, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
         "data": "synthetic (seeded N(0,1) weights ternarised on device; N(0,1) activations, 1% channels x20)",
+        "path": "bitnet_w2a8_linear per linear (activation quantisation fused into the GEMV)",
         "config": {"workload": WORKLOAD, "shapes_out_x_K": [[o, k] for _, o, k in SHAPES], "layers": LAYERS,
                    "batch": B, "linears_per_step": LAYERS * len(SHAPES),
                    "l2": "inputs larger than L2 (520 MB packed weights per step); per-shape passes flush L2",
-                   "graph": "the 240 C-ABI calls of a step captured in one CUDA graph",
+                   "graph": "the 120 C-ABI calls of a step captured in one CUDA graph",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
         "per_shape_gemv": per_shape,
+        "two_call_step": {"ms_per_step": round(two_ms_max, 4),
+                          "GB/s": round(aggregate([two_ms_max] * world, [gbytes + qbytes] * world)[0], 2),
+                          "launches_per_step": two_launches,
+                          "how": "bitnet_quant_act + bitnet_w2a8_gemv per linear, same graph replay timing"},
         "gemv_only_ms_per_step": round(gemv_ms_max, 4),
         "prefill": prefill,
         "roofline": roofline,
@@ -476,7 +509,7 @@ def run_reference(args, rank, world):
             r = max(1, int(frac_rows))
             q, s, _ = oracle.quant_act(x)
             oracle.linear(codes[:r], sc[:r], k, q, s)
-            nbytes += gemv_bytes(r, k) + 5 * k + 4
+            nbytes += linear_bytes(r, k)
         return nbytes
 
     t0 = time.perf_counter()
@@ -522,7 +555,7 @@ def cpu_baseline(seconds=12.0):
         sc = np.full((o, k // 128), g, dtype=np.float32)
         x = syn.activations(syn.seed_for(CONFIG_ID, 0, m, syn.KIND_ACT), B, k, outliers=True)
         cases.append((o, k, codes, sc, x))
-    per_layer = sum(gemv_bytes(o, k) + 5 * k + 4 for o, k, *_ in cases)
+    per_layer = sum(linear_bytes(o, k) for o, k, *_ in cases)
     t0 = time.perf_counter()
     n = 0
     while True:
@@ -538,16 +571,69 @@ def cpu_baseline(seconds=12.0):
             "us_per_layer": round(dt / n * 1e6, 1)}
 
 
+# ------------------------------------------------------- small cases --
+
+def run_case(args):
+    """One kernel on one shape, for profiling: `--case gemv` runs
+    bitnet_w2a8_gemv over `--copies` distinct weights (so the weights exceed
+    L2), `--case gemm` runs bitnet_w2a8_gemm on one weight; `--reps` passes,
+    plain launches (no graph).  Prints one JSON line with the median time."""
+    import torch
+
+    import ternary_weight_absmax_b200 as b
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    o, k = args.rows, args.cols
+    seed = 0xB17E7 ^ 0x5A5A
+    copies = args.copies if args.case == "gemv" else 1
+    ws = build_weights(b, torch, dev, copies, [("w", o, k)], seed)
+    T = args.batch if args.case == "gemv" else args.tokens
+    x = torch.randn(T * k, dtype=torch.float32, device=dev)
+    q = torch.empty(T * k, dtype=torch.int8, device=dev)
+    s = torch.empty(T, dtype=torch.float32, device=dev)
+    y = torch.empty(T * o, dtype=torch.float32, device=dev)
+    b.bitnet_quant_act(x, T, k, q, s)
+    call = b.bitnet_w2a8_gemv if args.case == "gemv" else b.bitnet_w2a8_gemm
+    times = []
+    for _ in range(args.reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for c in range(copies):
+            call(ws[(c, "w")], q, s, T, y)
+        e1.record()
+        e1.synchronize()
+        times.append(e0.elapsed_time(e1) * 1e3 / copies)
+    assert b.bitnet_get_device_error() == b.BITNET_OK
+    med = sorted(times)[len(times) // 2]
+    out = {"case": args.case, "out": o, "K": k, "T": T, "copies": copies, "us_per_launch": round(med, 3)}
+    if args.case == "gemv":
+        out["GB/s"] = round(gemv_bytes(o, k, T) / (med * 1e-6) / 1e9, 1)
+    else:
+        out["TOPS"] = round(2.0 * T * o * k / (med * 1e-6) / 1e12, 1)
+    print(json.dumps(out), flush=True)
+
+
 # ------------------------------------------------------------------ main --
 
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--case", choices=["gemv", "gemm"], help="profile one kernel on one shape")
+    ap.add_argument("--rows", type=int, default=13824)
+    ap.add_argument("--cols", type=int, default=2560)
+    ap.add_argument("--batch", type=int, default=1)
+    ap.add_argument("--tokens", type=int, default=2048)
+    ap.add_argument("--copies", type=int, default=16)
+    ap.add_argument("--reps", type=int, default=5)
     args = ap.parse_args()
+    if args.case:
+        run_case(args)
+        return
 
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))

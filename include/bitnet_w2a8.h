@@ -215,9 +215,24 @@ bitnet_status bitnet_quant_act(const float *x_dev, int64_t T, int64_t K, int8_t 
  * q_dev: B*K int8 (16-byte aligned); s_dev: B fp32; y_dev: B*rows fp32
  * (4-byte aligned).  The sum over blocks runs in fp64 and is rounded once.
  * Errors: NULL, SHAPE (B outside 1..16, K mismatch), ALIGN, VALUE (w not
- * repacked), CUDA. */
+ * repacked), CUDA.
+ * The GEMV, the fused linear and the quantiser use programmatic dependent
+ * launch: a GEMV may start reading its (constant) weights while the kernel
+ * before it on the stream is still running, and reads q, s (or x) and writes
+ * y only after that kernel has finished.  Weights are never written by the
+ * library's own kernels after bitnet_repack_device returns. */
 bitnet_status bitnet_w2a8_gemv(const bitnet_weight *w, const int8_t *q_dev, const float *s_dev,
                                int64_t B, float *y_dev, bitnet_stream_t stream);
+
+/* Decode linear layer in one kernel, 1 <= B <= 16: quantises fp32 x [B][K]
+ * exactly as bitnet_quant_act does, then computes what bitnet_w2a8_gemv
+ * computes, without a global round trip of q (every CTA re-quantises x into
+ * shared memory).  x_dev: B*K fp32 (16-byte aligned); y_dev: B*rows fp32.
+ * q_out_dev (B*K int8) and s_out_dev (B fp32) are optional (NULL = not
+ * written; 4-byte aligned) and receive the quantised activations.
+ * Errors: NULL, SHAPE, ALIGN, VALUE, BUFSIZE, CUDA. */
+bitnet_status bitnet_w2a8_linear(const bitnet_weight *w, const float *x_dev, int64_t B, float *y_dev,
+                                 int8_t *q_out_dev, float *s_out_dev, bitnet_stream_t stream);
 
 /* Prefill GEMM, T >= 1 tokens, same result as the GEMV (tcgen05 int8
  * tensor cores, int32 accumulators in tensor memory).
@@ -234,6 +249,9 @@ bitnet_status bitnet_w2a8_gemm(const bitnet_weight *w, const int8_t *q_dev, cons
 bitnet_status bitnet_w2a8_gemv_acc(const bitnet_weight *w, const int8_t *q_dev,
                                    const float *s_dev, int64_t B, float *y_dev,
                                    int32_t *acc_dev, bitnet_stream_t stream);
+bitnet_status bitnet_w2a8_linear_acc(const bitnet_weight *w, const float *x_dev, int64_t B, float *y_dev,
+                                     int8_t *q_out_dev, float *s_out_dev, int32_t *acc_dev,
+                                     bitnet_stream_t stream);
 bitnet_status bitnet_w2a8_gemm_acc(const bitnet_weight *w, const int8_t *q_dev,
                                    const float *s_dev, int64_t T, float *y_dev,
                                    int32_t *acc_dev, bitnet_stream_t stream);

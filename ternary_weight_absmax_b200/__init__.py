@@ -76,6 +76,8 @@ def _load() -> ctypes.CDLL:
         "bitnet_quant_act": ([vp, i64, i64, vp, vp, vp, vp], st),
         "bitnet_w2a8_gemv": ([W, vp, vp, i64, vp, vp], st),
         "bitnet_w2a8_gemm": ([W, vp, vp, i64, vp, vp], st),
+        "bitnet_w2a8_linear": ([W, vp, i64, vp, vp, vp, vp], st),
+        "bitnet_w2a8_linear_acc": ([W, vp, i64, vp, vp, vp, vp, vp], st),
         "bitnet_w2a8_gemv_acc": ([W, vp, vp, i64, vp, vp, vp], st),
         "bitnet_w2a8_gemm_acc": ([W, vp, vp, i64, vp, vp, vp], st),
         "bitnet_get_device_error": ([vp], st),
@@ -255,6 +257,22 @@ def bitnet_w2a8_gemv(w: Weight, q, s, B: int, y, stream=None):
 def bitnet_w2a8_gemm(w: Weight, q, s, T: int, y, stream=None):
     _check(_lib.bitnet_w2a8_gemm(w.ref(), _dptr(q, "int8", T * w.cols, "q"), _dptr(s, "float32", T, "s"), T,
                                  _dptr(y, "float32", T * w.rows, "y"), _stream(stream)), "bitnet_w2a8_gemm")
+
+
+def bitnet_w2a8_linear(w: Weight, x, B: int, y, q_out=None, s_out=None, stream=None):
+    """Fused act-quant + GEMV: fp32 x [B*K] -> y [B*rows]; optional q_out/s_out."""
+    _check(_lib.bitnet_w2a8_linear(w.ref(), _dptr(x, "float32", B * w.cols, "x"), B,
+                                   _dptr(y, "float32", B * w.rows, "y"), _dptr(q_out, "int8", B * w.cols, "q_out"),
+                                   _dptr(s_out, "float32", B, "s_out"), _stream(stream)), "bitnet_w2a8_linear")
+
+
+def bitnet_w2a8_linear_acc(w: Weight, x, B: int, y, acc, q_out=None, s_out=None, stream=None):
+    _check(_lib.bitnet_w2a8_linear_acc(w.ref(), _dptr(x, "float32", B * w.cols, "x"), B,
+                                       _dptr(y, "float32", B * w.rows, "y"),
+                                       _dptr(q_out, "int8", B * w.cols, "q_out"),
+                                       _dptr(s_out, "float32", B, "s_out"),
+                                       _dptr(acc, "int32", B * w.rows * (w.cols // QK), "acc"), _stream(stream)),
+           "bitnet_w2a8_linear_acc")
 
 
 def bitnet_w2a8_gemv_acc(w: Weight, q, s, B: int, y, acc, stream=None):

@@ -278,8 +278,37 @@ static bitnet_status gemv_impl(const bitnet_weight *w, const int8_t *q_dev, cons
     if (!aligned(q_dev, 16) || !aligned(s_dev, 4) || !aligned(y_dev, 4) || (acc_dev && !aligned(acc_dev, 4)))
         return fail(BITNET_ERR_ALIGN, "q needs 16-byte, s/y/acc 4-byte alignment");
     cudaError_t e = launch_gemv(w->data, w->rows, w->cols, (w->flags & BITNET_WEIGHT_UNIFORM_ROWS) != 0,
-                                q_dev, s_dev, B, y_dev, acc_dev, reinterpret_cast<cudaStream_t>(stream));
+                                q_dev, s_dev, B, y_dev, acc_dev, nullptr, nullptr, nullptr,
+                                reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? BITNET_OK : cuda_fail(e, "gemv launch");
+}
+
+static bitnet_status linear_impl(const bitnet_weight *w, const float *x_dev, int64_t B, float *y_dev,
+                                 int8_t *q_out_dev, float *s_out_dev, int32_t *acc_dev, bitnet_stream_t stream) {
+    t_detail[0] = 0;
+    bitnet_status s = check_weight(w);
+    if (s != BITNET_OK) return s;
+    if (B < 1 || B > 16) return fail(BITNET_ERR_SHAPE, "linear batch %lld outside 1..16", (long long)B);
+    if (!x_dev || !y_dev) return fail(BITNET_ERR_NULL, "NULL pointer");
+    if (!aligned(x_dev, 16) || !aligned(y_dev, 4) || (q_out_dev && !aligned(q_out_dev, 4)) ||
+        (s_out_dev && !aligned(s_out_dev, 4)) || (acc_dev && !aligned(acc_dev, 4)))
+        return fail(BITNET_ERR_ALIGN, "x needs 16-byte, y/q_out/s_out/acc 4-byte alignment");
+    cudaError_t e = launch_gemv(w->data, w->rows, w->cols, (w->flags & BITNET_WEIGHT_UNIFORM_ROWS) != 0,
+                                nullptr, nullptr, B, y_dev, acc_dev, x_dev, q_out_dev, s_out_dev,
+                                reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? BITNET_OK : cuda_fail(e, "linear launch");
+}
+
+bitnet_status bitnet_w2a8_linear(const bitnet_weight *w, const float *x_dev, int64_t B, float *y_dev,
+                                 int8_t *q_out_dev, float *s_out_dev, bitnet_stream_t stream) {
+    return linear_impl(w, x_dev, B, y_dev, q_out_dev, s_out_dev, nullptr, stream);
+}
+
+bitnet_status bitnet_w2a8_linear_acc(const bitnet_weight *w, const float *x_dev, int64_t B, float *y_dev,
+                                     int8_t *q_out_dev, float *s_out_dev, int32_t *acc_dev,
+                                     bitnet_stream_t stream) {
+    if (!acc_dev) return fail(BITNET_ERR_NULL, "acc is NULL");
+    return linear_impl(w, x_dev, B, y_dev, q_out_dev, s_out_dev, acc_dev, stream);
 }
 
 bitnet_status bitnet_w2a8_gemv(const bitnet_weight *w, const int8_t *q_dev, const float *s_dev, int64_t B,

@@ -70,9 +70,11 @@ cudaError_t launch_repack(const uint8_t *codes, const float *scales, int64_t row
                           void *data, cudaStream_t st);
 cudaError_t launch_unrepack(const void *data, int64_t rows, int64_t cols, uint8_t *codes,
                             float *scales, cudaStream_t st);
+// x non-null: the fused path (quantise x in the kernel; q, s ignored; q_out and
+// s_out, if non-null, receive the quantised activations).
 cudaError_t launch_gemv(const void *data, int64_t rows, int64_t cols, bool uniform,
                         const int8_t *q, const float *s, int64_t B, float *y, int32_t *acc,
-                        cudaStream_t st);
+                        const float *x, int8_t *q_out, float *s_out, cudaStream_t st);
 int absmean_num_partials(int64_t n);
 cudaError_t launch_ternarize(const float *w, int64_t rows, int64_t cols, bool per_block, uint32_t *codes,
                              float *scales, double *partials, float *gamma_slot, cudaStream_t st);

@@ -12,7 +12,8 @@
 // int8 per thread per step.  Each warp step covers 32 float4 = one 128-wide
 // block, so the optional per-block sums of q are one warp reduction each.
 // Bound: HBM for prefill-sized T (4 B read + 1 B written per element), launch
-// latency for decode.
+// latency for decode.  Launched with programmatic dependent launch so the
+// next kernel (the GEMV) can start streaming its weights meanwhile.
 #include "common.cuh"
 
 namespace bitnet {
@@ -33,6 +34,11 @@ template <bool kBlockSum>
 __global__ void __launch_bounds__(kThreads)
 quant_act_kernel(const float4 *__restrict__ x, int64_t K, int8_t *__restrict__ q,
                  float *__restrict__ s, int32_t *__restrict__ blocksum) {
+    // x may be produced by the kernel just before on the stream: wait for it
+    // (a no-op without programmatic dependent launch), then let the next
+    // kernel launch so it can prefetch its weights while this one runs.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int64_t row = blockIdx.x;
     const int64_t n4 = K / 4;
     const float4 *xr = x + row * n4;
@@ -83,14 +89,18 @@ quant_act_kernel(const float4 *__restrict__ x, int64_t K, int8_t *__restrict__ q
 cudaError_t launch_quant_act(const float *x, int64_t T, int64_t K, int8_t *q, float *s,
                              int32_t *blocksum, cudaStream_t st) {
     if (T == 0) return cudaSuccess;
-    dim3 grid((unsigned)T);
-    if (blocksum)
-        quant_act_kernel<true><<<grid, kThreads, 0, st>>>(reinterpret_cast<const float4 *>(x), K,
-                                                          q, s, blocksum);
-    else
-        quant_act_kernel<false><<<grid, kThreads, 0, st>>>(reinterpret_cast<const float4 *>(x), K,
-                                                           q, s, nullptr);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)T);
+    cfg.blockDim = dim3(kThreads);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const float4 *x4 = reinterpret_cast<const float4 *>(x);
+    if (blocksum) return cudaLaunchKernelEx(&cfg, quant_act_kernel<true>, x4, K, q, s, blocksum);
+    return cudaLaunchKernelEx(&cfg, quant_act_kernel<false>, x4, K, q, s, (int32_t *)nullptr);
 }
 
 }  // namespace bitnet

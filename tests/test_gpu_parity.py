@@ -346,3 +346,87 @@ def test_gemm_zero_tokens_is_a_no_op():
     b.bitnet_w2a8_gemm(w, q, s, 0, y)
     assert b.bitnet_get_device_error() == b.BITNET_OK
     assert np.all(to_np(y) == 5.0)
+
+
+# ---------------------------------------------------- fused decode linear --
+
+def _run_linear(t, sc, x, with_acc=False, guard=64):
+    b = lib()
+    tt = torch()
+    rows, K = t.shape
+    B = x.shape[0]
+    w, _ = device_weight(t, sc)
+    xd = cuda(x.astype(np.float32).reshape(-1))
+    ybuf = tt.full((B * rows + 2 * guard,), 12345.0, dtype=tt.float32, device="cuda")
+    y = ybuf[guard:guard + B * rows]
+    q = tt.full((B * K,), 99, dtype=tt.int8, device="cuda")
+    s = tt.full((B,), -1.0, dtype=tt.float32, device="cuda")
+    acc = None
+    if with_acc:
+        acc = tt.full((B * rows * (K // QK),), -7, dtype=tt.int32, device="cuda")
+        b.bitnet_w2a8_linear_acc(w, xd, B, y, acc, q, s)
+    else:
+        b.bitnet_w2a8_linear(w, xd, B, y, q, s)
+    yb = to_np(ybuf)
+    assert np.all(yb[:guard] == 12345.0) and np.all(yb[guard + B * rows:] == 12345.0), "output guard overwritten"
+    return to_np(q).reshape(B, K), to_np(s), to_np(y).reshape(B, rows), \
+        (to_np(acc).reshape(B, rows, K // QK) if acc is not None else None)
+
+
+@pytest.mark.parametrize("rows,K,B,mode", [
+    (256, 512, 1, "tensor"), (256, 512, 1, "block"), (1, 128, 1, "tensor"), (17, 128, 16, "block"),
+    (1000, 640, 3, "block"), (3840, 2560, 1, "tensor"), (2560, 6912, 1, "tensor"), (2560, 2560, 16, "tensor"),
+    (777, 1280, 8, "row"), (4096, 14336, 4, "tensor"), (2560, 14336, 16, "block"),
+])
+def test_linear_matches_oracle_and_gemv(rows, K, B, mode):
+    t, sc, x = _gemv_case(rows, K, B, mode, seed=rows * 13 + K + B)
+    q, s, y, acc = _run_linear(t, sc, x, with_acc=True)
+    rq, rs, _ = oracle.quant_act(x)
+    np.testing.assert_array_equal(q, rq)
+    np.testing.assert_array_equal(s.view(np.uint32), rs.view(np.uint32))
+    np.testing.assert_array_equal(acc, oracle.block_acc(oracle.pack_i2s(t), K, rq))
+    ref = oracle.linear(oracle.pack_i2s(t), sc, K, rq, rs)
+    assert_close(y, ref, f"linear {rows}x{K} B={B} {mode}")
+    if mode != "block":
+        np.testing.assert_array_equal(y, ref)
+    _, _, _, _, yg, _ = _run_gemv(t, sc, x)            # same arithmetic as quant_act + gemv
+    np.testing.assert_array_equal(y, yg)
+    q2, s2, y2, _ = _run_linear(t, sc, x)              # plain entry point
+    np.testing.assert_array_equal(y2, y)
+
+
+@pytest.mark.parametrize("B", list(range(1, 17)))
+def test_linear_every_batch_size(B):
+    rows, K = 300, 1024
+    t, sc, x = _gemv_case(rows, K, B, "tensor", seed=1700 + B)
+    q, s, y, _ = _run_linear(t, sc, x)
+    rq, rs, _ = oracle.quant_act(x)
+    np.testing.assert_array_equal(q, rq)
+    np.testing.assert_array_equal(y, oracle.linear(oracle.pack_i2s(t), sc, K, rq, rs))
+
+
+def test_linear_optional_outputs_and_zero_rows():
+    b = lib()
+    tt = torch()
+    rows, K, B = 64, 512, 3
+    t, sc, x = _gemv_case(rows, K, B, "tensor", seed=91)
+    x[1] = 0.0
+    w, _ = device_weight(t, sc)
+    y = tt.empty(B * rows, dtype=tt.float32, device="cuda")
+    b.bitnet_w2a8_linear(w, cuda(x.reshape(-1)), B, y)            # no q/s outputs
+    rq, rs, _ = oracle.quant_act(x)
+    got = to_np(y).reshape(B, rows)
+    np.testing.assert_array_equal(got, oracle.linear(oracle.pack_i2s(t), sc, K, rq, rs))
+    assert np.all(got[1] == 0.0)
+
+
+@pytest.mark.parametrize("rows,K", [(3840, 2560), (13824, 2560), (2560, 6912), (28672, 4096), (4096, 14336)])
+@pytest.mark.parametrize("B", [1, 16])
+def test_linear_full_size_sampled_rows(rows, K, B):
+    t, sc, x = _gemv_case(rows, K, B, "tensor", seed=rows + 3 * K + B)
+    q, s, y, _ = _run_linear(t, sc, x)
+    rq, rs, _ = oracle.quant_act(x)
+    np.testing.assert_array_equal(q, rq)
+    pick = np.unique(np.concatenate([[0, rows - 1], syn.splitmix64(rows ^ B, np.arange(40)) % np.uint64(rows)]))
+    pick = pick.astype(np.int64)
+    np.testing.assert_array_equal(y[:, pick], oracle.linear(oracle.pack_i2s(t[pick]), sc[pick], K, rq, rs))
