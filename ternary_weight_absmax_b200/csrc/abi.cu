@@ -89,6 +89,18 @@ cudaError_t device_globals(DeviceGlobals *out) {
     return cudaSuccess;
 }
 
+int num_sms() {
+    static int n[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (!n[dev]) {
+        int v = 0;
+        if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) v = 148;
+        n[dev] = v;
+    }
+    return n[dev];
+}
+
 }  // namespace bitnet
 
 using namespace bitnet;
@@ -277,9 +289,11 @@ static bitnet_status gemv_impl(const bitnet_weight *w, const int8_t *q_dev, cons
     if (!q_dev || !s_dev || !y_dev) return fail(BITNET_ERR_NULL, "NULL pointer");
     if (!aligned(q_dev, 16) || !aligned(s_dev, 4) || !aligned(y_dev, 4) || (acc_dev && !aligned(acc_dev, 4)))
         return fail(BITNET_ERR_ALIGN, "q needs 16-byte, s/y/acc 4-byte alignment");
-    cudaError_t e = launch_gemv(w->data, w->rows, w->cols, (w->flags & BITNET_WEIGHT_UNIFORM_ROWS) != 0,
-                                q_dev, s_dev, B, y_dev, acc_dev, nullptr, nullptr, nullptr,
-                                reinterpret_cast<cudaStream_t>(stream));
+    DeviceGlobals g;
+    cudaError_t e = device_globals(&g);
+    if (e != cudaSuccess) return cuda_fail(e, "device globals");
+    e = launch_gemv(w->data, w->rows, w->cols, (w->flags & BITNET_WEIGHT_UNIFORM_ROWS) != 0, q_dev, s_dev, B,
+                    y_dev, acc_dev, nullptr, nullptr, nullptr, g, reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? BITNET_OK : cuda_fail(e, "gemv launch");
 }
 
@@ -293,9 +307,11 @@ static bitnet_status linear_impl(const bitnet_weight *w, const float *x_dev, int
     if (!aligned(x_dev, 16) || !aligned(y_dev, 4) || (q_out_dev && !aligned(q_out_dev, 4)) ||
         (s_out_dev && !aligned(s_out_dev, 4)) || (acc_dev && !aligned(acc_dev, 4)))
         return fail(BITNET_ERR_ALIGN, "x needs 16-byte, y/q_out/s_out/acc 4-byte alignment");
-    cudaError_t e = launch_gemv(w->data, w->rows, w->cols, (w->flags & BITNET_WEIGHT_UNIFORM_ROWS) != 0,
-                                nullptr, nullptr, B, y_dev, acc_dev, x_dev, q_out_dev, s_out_dev,
-                                reinterpret_cast<cudaStream_t>(stream));
+    DeviceGlobals g;
+    cudaError_t e = device_globals(&g);
+    if (e != cudaSuccess) return cuda_fail(e, "device globals");
+    e = launch_gemv(w->data, w->rows, w->cols, (w->flags & BITNET_WEIGHT_UNIFORM_ROWS) != 0, nullptr, nullptr, B,
+                    y_dev, acc_dev, x_dev, q_out_dev, s_out_dev, g, reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? BITNET_OK : cuda_fail(e, "linear launch");
 }
 

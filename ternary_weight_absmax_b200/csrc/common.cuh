@@ -63,6 +63,9 @@ struct DeviceGlobals {
 };
 cudaError_t device_globals(DeviceGlobals *out);
 
+// Streaming multiprocessors of the current device (cached per device).
+int num_sms();
+
 // Launchers (return the launch error, if any).
 cudaError_t launch_quant_act(const float *x, int64_t T, int64_t K, int8_t *q, float *s,
                              int32_t *blocksum, cudaStream_t st);
@@ -74,7 +77,14 @@ cudaError_t launch_unrepack(const void *data, int64_t rows, int64_t cols, uint8_
 // s_out, if non-null, receive the quantised activations).
 cudaError_t launch_gemv(const void *data, int64_t rows, int64_t cols, bool uniform,
                         const int8_t *q, const float *s, int64_t B, float *y, int32_t *acc,
-                        const float *x, int8_t *q_out, float *s_out, cudaStream_t st);
+                        const float *x, int8_t *q_out, float *s_out, const DeviceGlobals &g,
+                        cudaStream_t st);
+// Batch-1 decode kernel for uniform rows (decode.cu); launch_gemv picks it when
+// decode_b1_supported says it takes the shape.
+bool decode_b1_supported(int64_t rows, int64_t cols, bool fused);
+cudaError_t launch_decode_b1(const void *data, int64_t rows, int64_t cols, const int8_t *q, const float *s,
+                             float *y, const float *x, int8_t *q_out, float *s_out, const DeviceGlobals &g,
+                             cudaStream_t st);
 int absmean_num_partials(int64_t n);
 cudaError_t launch_ternarize(const float *w, int64_t rows, int64_t cols, bool per_block, uint32_t *codes,
                              float *scales, double *partials, float *gamma_slot, cudaStream_t st);

@@ -1,0 +1,387 @@
+// decode.cu -- batch-1 W2A8 linear for uniform rows (the per-tensor absmean
+// case): the latency-critical call of token-by-token generation.
+//
+// y[o] = rowscale[o] * (sum_k t[o][k] * q[k]) / s,   q = per-token absmax int8
+// activations ("5倍性能跃升：BitNet与llama.cpp的1-bit LLM推理架构对决", section
+// "GPU内核突破": 2-bit weights x 8-bit activations with dp4a; the activation
+// quantisation is the per-token absmax of "BitNet b1.58", section "Quantization
+// Function").  The arithmetic is that of the general GEMV kernel: integer dot
+// products, one exact fp64 product with the row scale, one fp64 divide by s,
+// one rounding to fp32.
+//
+// A decode step is a chain of dependent linears of a few microseconds each, so
+// what costs is the chain's latency: the time from the previous kernel's end
+// to this kernel's last store.  Measured on B200, the pieces of that are the
+// release of griddepcontrol.wait (~0.5 us after the previous grid ends), one
+// L2 round trip for x, the CTA barriers and the dp4a work; weights that are
+// still in flight when the products start add their DRAM time on top.  Hence:
+//
+//  * one CTA of 16 warps per SM with less than half of the SM's registers and
+//    shared memory, so that the next linear's CTAs are resident while this one
+//    runs (programmatic dependent launch) and fetch their weights before their
+//    griddepcontrol.wait;
+//  * the weights move by bulk copies (cp.async.bulk, one per two 512-byte
+//    tiles, L2 evict-first: they are read once per step and must not push the
+//    activations out of L2) into shared memory, up to eight tiles per warp in
+//    flight; register loads could not keep enough bytes in flight per SM;
+//  * a CTA owns whole row tiles (no cross-CTA reduction) and its warps split
+//    the (tile, block) items evenly in memory order, so a warp's tiles are one
+//    contiguous range;
+//  * after the wait: x is read once into registers, the absmax is combined
+//    across warps through shared memory (one barrier), x is quantised into
+//    shared memory in the order the lanes read it (a lane's eight words of a
+//    block are 32 contiguous bytes) and sum(q) is taken once per CTA (second
+//    barrier); then the masked dp4a products, one shared-memory atomic per row
+//    and tile change, the third barrier and the epilogue.
+// Integer sums are exact, so the atomics leave the result independent of
+// their order.  Every wait on a copy is bounded; on a timeout the kernel sets
+// the device error word, waits (bounded) for its copies in flight and returns.
+#include "common.cuh"
+#include "dp4a.cuh"
+#include "tcgen05.cuh"
+
+namespace bitnet {
+namespace {
+
+constexpr int kWarps = 16;
+constexpr int kThreads = kWarps * 32;
+constexpr int kChunk = 2;     // tiles per bulk copy
+constexpr int kMaxSlots = 4;  // copies in flight per warp
+constexpr int kTile = kTileBytes;
+constexpr uint32_t kDrainLimit = 1u << 26;  // tries while waiting out a copy after a timeout
+
+struct DecArgs {
+    const unsigned char *tiles;
+    const float *rowscale;
+    const int8_t *q;   // [K] (unfused)
+    const float *s;    // [1] (unfused)
+    const float *x;    // [K] fp32 (fused)
+    int8_t *q_out;     // nullable (fused): written by CTA 0
+    float *s_out;      // nullable (fused): written by CTA 0
+    float *y;
+    unsigned *err;
+    const unsigned *wait_limit;
+    int64_t rows;
+    int K;
+    int nb;
+    int tiles_lo;  // every CTA owns tiles_lo or tiles_lo + 1 row tiles
+    int extra;     // the first `extra` CTAs own tiles_lo + 1
+    int wcap;      // tiles of shared memory per warp: kChunk * (copies in flight)
+    uint32_t off_q, off_acc, off_rsc, off_red, off_bar;
+};
+
+// Shared-memory word of activation word m (bytes 4m .. 4m+3 of q): lane-part t
+// of block j, slot 2*group + half, so that lane t's words qa0 qb0 qa1 qb1 qa2
+// qb2 qa3 qb3 of a block are contiguous.
+__device__ __forceinline__ int perm_word(int m) {
+    const int w = m & 31;
+    return (m & ~31) | ((w & 3) << 3) | ((w >> 3) << 1) | ((w >> 2) & 1);
+}
+
+// Lane 0 waits on the mbarrier phase (bounded), the warp gets the verdict.
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, uint32_t limit) {
+    int ok = 0;
+    if ((threadIdx.x & 31) == 0) ok = ptx::mbar_wait(bar, parity, limit, nullptr) ? 1 : 0;
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    return ok != 0;
+}
+
+template <bool FUSED, int NX>
+__global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const DecArgs a) {
+    extern __shared__ __align__(128) unsigned char smem[];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int g = lane >> 2, t = lane & 3;
+    const int c = blockIdx.x;
+    const int64_t r0 = (int64_t)c * a.tiles_lo + min(c, a.extra);
+    const int nr = a.tiles_lo + (c < a.extra ? 1 : 0);
+    const int n = nr * a.nb;
+    const int i0 = (int)(((int64_t)warp * n) / kWarps);
+    const int nit = (int)(((int64_t)(warp + 1) * n) / kWarps) - i0;
+    const int nslots = a.wcap / kChunk;
+    const int nchunks = (nit + kChunk - 1) / kChunk;
+    unsigned char *wsm = smem + (size_t)warp * a.wcap * kTile;
+    uint32_t *qw = reinterpret_cast<uint32_t *>(smem + a.off_q);
+    int *acc = reinterpret_cast<int *>(smem + a.off_acc);
+    float *rsc = reinterpret_cast<float *>(smem + a.off_rsc);
+    unsigned *wmax = reinterpret_cast<unsigned *>(smem + a.off_red);
+    int *wqs = reinterpret_cast<int *>(smem + a.off_red + 64);
+    const uint32_t bars = ptx::smem_u32(smem + a.off_bar) + 8u * (warp * kMaxSlots);
+    const uint32_t rbar = ptx::smem_u32(smem + a.off_bar) + 8u * (kWarps * kMaxSlots);
+    const unsigned char *src = a.tiles + (size_t)(r0 * a.nb + i0) * kTile;
+    const uint32_t limit = *a.wait_limit;
+
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
+    // ---- before the wait: nothing here depends on the previous kernel.
+    const uint64_t pol = ptx::policy_evict_first();
+    auto issue = [&](int k) {  // lane 0: chunk k of this warp's tiles into its slot
+        const int s = k % nslots;
+        const uint32_t bytes = (uint32_t)min(kChunk, nit - k * kChunk) * kTile;
+        ptx::mbar_arrive_expect_tx(bars + 8u * s, bytes);
+        ptx::bulk_g2s(ptx::smem_u32(wsm + s * kChunk * kTile), src + (size_t)k * kChunk * kTile, bytes,
+                      bars + 8u * s, pol);
+    };
+    if (lane == 0) {
+        for (int s = 0; s < nslots; s++) ptx::mbar_init(bars + 8u * s, 1);
+        if (warp == 0) ptx::mbar_init(rbar, 1);
+        ptx::fence_mbar_init();
+        for (int k = 0; k < nchunks && k < nslots; k++) issue(k);
+        if (warp == 0) {
+            const uint32_t bytes = (uint32_t)nr * kTileRows * sizeof(float);
+            ptx::mbar_arrive_expect_tx(rbar, bytes);
+            ptx::bulk_g2s(ptx::smem_u32(rsc), a.rowscale + r0 * kTileRows, bytes, rbar, pol);
+        }
+    }
+    for (int i = tid; i < nr * kTileRows; i += kThreads) acc[i] = 0;
+
+    asm volatile("griddepcontrol.wait;" ::: "memory");  // x (or q, s) ready; y free
+
+    // ---- activations: s, q (permuted) in shared memory, sum(q).
+    const int K4 = a.K >> 2;
+    float s;
+    int qsum = 0;
+    if constexpr (FUSED) {
+        const float4 *x4 = reinterpret_cast<const float4 *>(a.x);
+        float4 xv[NX];
+        float m = 0.0f;
+#pragma unroll
+        for (int u = 0; u < NX; u++) {
+            const int i = tid + u * kThreads;
+            xv[u] = i < K4 ? x4[i] : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+            m = fmaxf(m, fmaxf(fmaxf(fabsf(xv[u].x), fabsf(xv[u].y)), fmaxf(fabsf(xv[u].z), fabsf(xv[u].w))));
+        }
+        // m >= 0 and not NaN (fmaxf drops NaN): its bit pattern orders like its value.
+        const unsigned mu = __reduce_max_sync(0xffffffffu, __float_as_uint(m));
+        if (lane == 0) wmax[warp] = mu;
+        __syncthreads();
+        unsigned mm = 0u;
+#pragma unroll
+        for (int k = 0; k < kWarps / 4; k++) {
+            const uint4 v = reinterpret_cast<const uint4 *>(wmax)[k];
+            mm = max(mm, max(max(v.x, v.y), max(v.z, v.w)));
+        }
+        const float amax = __uint_as_float(mm);
+        s = __fdiv_rn(127.0f, amax > kEps ? amax : kEps);
+        if (c == 0 && tid == 0 && a.s_out) a.s_out[0] = s;
+        uint32_t *qo = (c == 0 && a.q_out) ? reinterpret_cast<uint32_t *>(a.q_out) : nullptr;
+#pragma unroll
+        for (int u = 0; u < NX; u++) {
+            const int i = tid + u * kThreads;
+            if (i < K4) {
+                const uint32_t w = quant4(xv[u], s);
+                qw[perm_word(i)] = w;
+                qsum = dp4a_ss((int)w, 0x01010101, qsum);
+                if (qo) qo[i] = w;
+            }
+        }
+    } else {
+        s = *a.s;
+        const uint32_t *q4 = reinterpret_cast<const uint32_t *>(a.q);
+        for (int i = tid; i < K4; i += kThreads) {
+            const uint32_t w = q4[i];
+            qw[perm_word(i)] = w;
+            qsum = dp4a_ss((int)w, 0x01010101, qsum);
+        }
+    }
+    qsum = __reduce_add_sync(0xffffffffu, qsum);
+    if (lane == 0) wqs[warp] = qsum;
+    __syncthreads();
+
+    // ---- products.  Items of this warp: i0 .. i0 + nit - 1, tile r = i / nb,
+    // block j = i % nb; the four group sums of rows g and g + 8 are held until
+    // the tile changes.
+    int aA[4] = {0, 0, 0, 0}, aB[4] = {0, 0, 0, 0};
+    const int r = i0 / a.nb;
+    int j = i0 - r * a.nb;
+    int *accp = acc + r * kTileRows + g;  // rows g and g + 8 of the current tile
+    auto flush = [&]() {
+        const int pA = tig_reduce(combine4(aA));
+        const int pB = tig_reduce(combine4(aB));
+        if (t == 0) {
+            atomicAdd(accp, pA);
+            atomicAdd(accp + 8, pB);
+        }
+#pragma unroll
+        for (int k = 0; k < 4; k++) aA[k] = aB[k] = 0;
+    };
+    int k = 0;
+    bool ok = true;
+    for (; k < nchunks; k++) {
+        const int slot = k % nslots;
+        if (!warp_wait(bars + 8u * slot, (uint32_t)(k / nslots) & 1u, limit)) {
+            ok = false;
+            break;
+        }
+        const uint4 *cw = reinterpret_cast<const uint4 *>(wsm + slot * kChunk * kTile) + lane;
+        const int m = min(kChunk, nit - k * kChunk);
+#pragma unroll
+        for (int e = 0; e < kChunk; e++) {
+            if (e >= m) break;
+            const uint4 w = cw[e * 32];
+            const uint4 *qp = reinterpret_cast<const uint4 *>(qw + j * 32 + t * 8);
+#pragma unroll
+            for (int h = 0; h < 2; h++) {
+                const uint4 qv = qp[h];  // qa, qb of groups 2h and 2h + 1
+#pragma unroll
+                for (int f = 0; f < 2; f++) {
+                    const int gg = 2 * h + f;
+                    const int qa = (int)(f ? qv.z : qv.x), qb = (int)(f ? qv.w : qv.y);
+                    const uint32_t mk = 0xC0C0C0C0u >> (2 * gg);
+                    aA[gg] = dp4a_us(w.x & mk, qa, aA[gg]);
+                    aA[gg] = dp4a_us(w.z & mk, qb, aA[gg]);
+                    aB[gg] = dp4a_us(w.y & mk, qa, aB[gg]);
+                    aB[gg] = dp4a_us(w.w & mk, qb, aB[gg]);
+                }
+            }
+            if (++j == a.nb) {
+                flush();
+                accp += kTileRows;
+                j = 0;
+            }
+        }
+        if (k + nslots < nchunks) {
+            __syncwarp();  // every lane has read the slot
+            if (lane == 0) {
+                ptx::fence_proxy_async_smem();
+                issue(k + nslots);
+            }
+        }
+    }
+    if (!ok) {
+        // Timed out: record it, then wait out this warp's copies still in flight.
+        if (lane == 0) {
+            atomicOr(a.err, kErrTimeout);
+            for (int kk = k; kk < nchunks && kk < k + nslots; kk++)
+                ptx::mbar_wait(bars + 8u * (kk % nslots), (uint32_t)(kk / nslots) & 1u, kDrainLimit, nullptr);
+        }
+        __syncwarp();
+    }
+    if (j != 0) flush();  // items since the last tile change (none if j == 0)
+    if (warp == 0 && !warp_wait(rbar, 0u, limit)) {
+        if (lane == 0) {
+            atomicOr(a.err, kErrTimeout);
+            ptx::mbar_wait(rbar, 0u, kDrainLimit, nullptr);
+        }
+        __syncwarp();
+    }
+    __syncthreads();
+
+    // ---- epilogue: y = rowscale * (sum c*q - sum q) / s, fp64, one rounding.
+    int tot = 0;
+#pragma unroll
+    for (int w = 0; w < kWarps / 4; w++) {
+        const int4 v = reinterpret_cast<const int4 *>(wqs)[w];
+        tot += v.x + v.y + v.z + v.w;
+    }
+    for (int i = tid; i < nr * kTileRows; i += kThreads) {
+        const int64_t o = r0 * kTileRows + i;
+        if (o < a.rows) a.y[o] = (float)((double)rsc[i] * (double)(acc[i] - tot) / (double)s);
+    }
+}
+
+struct Plan {
+    int grid, nx, wcap;
+    size_t smem;
+    DecArgs a;
+};
+
+// Shapes, grid and shared-memory layout; false if the kernel does not take the
+// shape (the general kernel does).
+bool plan(const Layout &L, bool fused, Plan *p) {
+    const int sms = num_sms();
+    const int grid = (int)(L.ntr < sms ? L.ntr : sms);
+    const int K = (int)L.cols;
+    int nx = 1;
+    while (nx * 4 * kThreads < K) nx *= 2;
+    if (fused && nx > 8) return false;
+    const int64_t lo = L.ntr / grid, hi = lo + (L.ntr % grid ? 1 : 0);
+    const int64_t per_warp = (hi * L.nb + kWarps - 1) / kWarps;
+    int wcap = (int)(per_warp < kChunk * kMaxSlots ? per_warp : kChunk * kMaxSlots);
+    wcap = (wcap + kChunk - 1) / kChunk * kChunk;
+    if (wcap < kChunk) wcap = kChunk;
+    DecArgs &a = p->a;
+    a.off_q = (uint32_t)(kWarps * wcap * kTile);
+    a.off_acc = (uint32_t)align_up(a.off_q + (size_t)K, 16);
+    a.off_rsc = a.off_acc + (uint32_t)(hi * kTileRows * sizeof(int));
+    a.off_red = a.off_rsc + (uint32_t)(hi * kTileRows * sizeof(float));
+    a.off_bar = a.off_red + 128;
+    const size_t smem = a.off_bar + 8 * (kWarps * kMaxSlots + 1);
+    if (smem > 100 * 1024) return false;  // two CTAs per SM
+    a.rows = L.rows;
+    a.K = K;
+    a.nb = (int)L.nb;
+    a.tiles_lo = (int)lo;
+    a.extra = (int)(L.ntr % grid);
+    a.wcap = wcap;
+    p->grid = grid;
+    p->nx = nx;
+    p->wcap = wcap;
+    p->smem = smem;
+    return true;
+}
+
+template <bool FUSED, int NX>
+cudaError_t run(const Plan &p, cudaStream_t st) {
+    auto k = decode_b1_kernel<FUSED, NX>;
+    static bool configured[64];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (!configured[dev]) {
+        // Every launch asks for the same shared-memory carveout, so CTAs of
+        // consecutive linears can share an SM without it being reconfigured.
+        e = cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, 100 * 1024);
+        if (e != cudaSuccess) return e;
+        configured[dev] = true;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)p.grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = p.smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, k, p.a);
+}
+
+}  // namespace
+
+bool decode_b1_supported(int64_t rows, int64_t cols, bool fused) {
+    Plan p;
+    return plan(layout_of(rows, cols), fused, &p);
+}
+
+cudaError_t launch_decode_b1(const void *data, int64_t rows, int64_t cols, const int8_t *q, const float *s,
+                             float *y, const float *x, int8_t *q_out, float *s_out, const DeviceGlobals &g,
+                             cudaStream_t st) {
+    const Layout L = layout_of(rows, cols);
+    Plan p;
+    if (!plan(L, x != nullptr, &p)) return cudaErrorNotSupported;
+    const unsigned char *base = static_cast<const unsigned char *>(data);
+    DecArgs &a = p.a;
+    a.tiles = base + L.off_tiles;
+    a.rowscale = reinterpret_cast<const float *>(base + L.off_rowscale);
+    a.q = q;
+    a.s = s;
+    a.x = x;
+    a.q_out = q_out;
+    a.s_out = s_out;
+    a.y = y;
+    a.err = g.err;
+    a.wait_limit = g.wait_limit;
+    if (!x) return run<false, 1>(p, st);
+    switch (p.nx) {
+        case 1: return run<true, 1>(p, st);
+        case 2: return run<true, 2>(p, st);
+        case 4: return run<true, 4>(p, st);
+        default: return run<true, 8>(p, st);
+    }
+}
+
+}  // namespace bitnet

@@ -425,18 +425,6 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
-int num_sms() {
-    static int n[64];
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-    if (!n[dev]) {
-        int v = 0;
-        if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) v = 148;
-        n[dev] = v;
-    }
-    return n[dev];
-}
-
 template <int BN, bool BLOCKWISE, bool ACC>
 cudaError_t run(const void *data, const Layout &L, const int8_t *q, GemmArgs a, cudaStream_t st) {
     using C = Cfg<BN, BLOCKWISE>;

@@ -36,6 +36,7 @@
 //  * Cross-lane and cross-warp reductions run in a fixed order, so results
 //    are deterministic.
 #include "common.cuh"
+#include "dp4a.cuh"
 
 namespace bitnet {
 namespace {
@@ -44,36 +45,6 @@ constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
 constexpr int kQSmemBudget = 32 * 1024;  // bytes of activations staged per K tile
 constexpr int kDepth = 8;                // weight loads in flight per lane
-
-__device__ __forceinline__ int dp4a_us(uint32_t a, int b, int c) {
-    int d;
-    asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
-    return d;
-}
-
-__device__ __forceinline__ int dp4a_ss(int a, int b, int c) { return __dp4a(a, b, c); }
-
-// Streaming 16-byte load of weights (read once: bypass L1).  volatile keeps the
-// compiler from sinking it below griddepcontrol.wait.
-__device__ __forceinline__ uint4 ld_stream(const uint4 *p) {
-    uint4 v;
-    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "l"(p));
-    return v;
-}
-
-// Four masked-and-scaled group sums -> sum of code*q.
-__device__ __forceinline__ int combine4(const int a[4]) {
-    return a[3] + (a[2] >> 2) + (a[1] >> 4) + (a[0] >> 6);
-}
-
-template <typename T>
-__device__ __forceinline__ T tig_reduce(T v) {
-    v += __shfl_xor_sync(0xffffffffu, v, 1);
-    v += __shfl_xor_sync(0xffffffffu, v, 2);
-    return v;
-}
 
 struct Args {
     const uint4 *tiles;
@@ -124,7 +95,7 @@ __device__ __forceinline__ void stage_q(const Args &a, int8_t *qs, int kt, int n
     for (int idx = threadIdx.x; idx < BT * per_row; idx += kThreads) {
         const int b = idx / per_row, c = idx - b * per_row;
         uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (b < a.B) v = __ldg(reinterpret_cast<const uint4 *>(a.q + (int64_t)b * a.K + kt) + c);
+        if (b < a.B) v = reinterpret_cast<const uint4 *>(a.q + (int64_t)b * a.K + kt)[c];
         reinterpret_cast<uint4 *>(qs + b * a.KT)[c] = v;
     }
 }
@@ -142,7 +113,7 @@ __device__ __forceinline__ void fused_scales(const Args &a, float *s_sh, float *
         if (b < a.B) {
             const float4 *xr = reinterpret_cast<const float4 *>(a.x + (int64_t)b * a.K);
             for (int i = threadIdx.x; i < n4; i += kThreads) {
-                const float4 v = __ldg(xr + i);
+                const float4 v = xr[i];
                 m = fmaxf(m, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
             }
         }
@@ -162,15 +133,6 @@ __device__ __forceinline__ void fused_scales(const Args &a, float *s_sh, float *
     __syncthreads();
 }
 
-__device__ __forceinline__ uint32_t quant4(float4 v, float s) {
-    auto one = [&](float x) {
-        int q = __float2int_rn(__fmul_rn(x, s));
-        q = q > 127 ? 127 : (q < -127 ? -127 : q);
-        return (uint32_t)(q & 0xff);
-    };
-    return one(v.x) | (one(v.y) << 8) | (one(v.z) << 16) | (one(v.w) << 24);
-}
-
 // Fused activation quantisation, pass 2: q[b][kt, kt+n) into the staged tile
 // (zero rows for b >= B); CTA 0 also writes q to q_out.
 template <int BT>
@@ -186,7 +148,7 @@ __device__ __forceinline__ void fused_stage_q(const Args &a, int8_t *qs, const f
                                ? reinterpret_cast<uint32_t *>(a.q_out + (int64_t)b * a.K + kt)
                                : nullptr;
             for (int i = threadIdx.x; i < n4; i += kThreads) {
-                const uint32_t w = quant4(__ldg(xr + i), sc);
+                const uint32_t w = quant4(xr[i], sc);
                 dst[i] = w;
                 if (qo) qo[i] = w;
             }
@@ -503,9 +465,12 @@ cudaError_t dispatch(Args &a, cudaStream_t st) {
 
 cudaError_t launch_gemv(const void *data, int64_t rows, int64_t cols, bool uniform,
                         const int8_t *q, const float *s, int64_t B, float *y, int32_t *acc,
-                        const float *x, int8_t *q_out, float *s_out, cudaStream_t st) {
+                        const float *x, int8_t *q_out, float *s_out, const DeviceGlobals &g,
+                        cudaStream_t st) {
     const Layout L = layout_of(rows, cols);
     const char *base = static_cast<const char *>(data);
+    if (B == 1 && uniform && !acc && decode_b1_supported(rows, cols, x != nullptr))
+        return launch_decode_b1(data, rows, cols, q, s, y, x, q_out, s_out, g, st);
     Args a;
     a.tiles = reinterpret_cast<const uint4 *>(base + L.off_tiles);
     a.tscales = reinterpret_cast<const float *>(base + L.off_tscales);

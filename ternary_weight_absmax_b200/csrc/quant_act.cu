@@ -89,6 +89,21 @@ quant_act_kernel(const float4 *__restrict__ x, int64_t K, int8_t *__restrict__ q
 cudaError_t launch_quant_act(const float *x, int64_t T, int64_t K, int8_t *q, float *s,
                              int32_t *blocksum, cudaStream_t st) {
     if (T == 0) return cudaSuccess;
+    static bool configured[64];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (!configured[dev]) {
+        // Same shared-memory carveout as the decode kernel, so the two can share
+        // an SM under programmatic dependent launch without a reconfiguration.
+        for (auto k : {quant_act_kernel<true>, quant_act_kernel<false>}) {
+            e = cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                     cudaSharedmemCarveoutMaxShared);
+            if (e != cudaSuccess) return e;
+        }
+        configured[dev] = true;
+    }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)T);
     cfg.blockDim = dim3(kThreads);

@@ -1,7 +1,8 @@
 // tcgen05.cuh -- thin inline-PTX wrappers for the sm_100a features the
-// prefill GEMM uses: mbarriers with bounded waits, TMA tensor loads (no
-// multicast), tensor-memory allocation, tcgen05.mma kind::i8, commits and
-// tensor-memory loads.  Written from the PTX ISA's instruction descriptions.
+// prefill GEMM and the decode kernel use: mbarriers with bounded waits, TMA
+// tensor loads and bulk copies (no multicast), tensor-memory allocation,
+// tcgen05.mma kind::i8, commits and tensor-memory loads.  Written from the PTX
+// ISA's instruction descriptions.
 #pragma once
 
 #include <cuda.h>
@@ -78,6 +79,24 @@ __device__ __forceinline__ bool mbar_wait_sleep(uint32_t bar, uint32_t parity, u
         __nanosleep(ns);
     }
     return false;
+}
+
+// Bulk copy global -> shared (no tensor map), completes on an mbarrier; the
+// L2 policy comes from createpolicy.  Addresses 16-byte aligned, size a
+// multiple of 16.
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar,
+                                         uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], "
+        "%4;" ::"r"(dst),
+        "l"((uint64_t)src), "r"(bytes), "r"(bar), "l"(policy)
+        : "memory");
+}
+// L2 policy: lines fetched with it are the first candidates for eviction.
+__device__ __forceinline__ uint64_t policy_evict_first() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
 }
 
 // TMA tensor store, shared -> global, tracked by bulk-async groups.

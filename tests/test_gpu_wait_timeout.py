@@ -37,3 +37,35 @@ def test_gemm_wait_timeout_is_reported_and_recoverable():
     assert b.bitnet_get_device_error() == b.BITNET_OK
     rq, rs, _ = oracle.quant_act(x)
     assert_close(to_np(y).reshape(T, rows), oracle.linear(oracle.pack_i2s(t), sc, K, rq, rs), "after timeout")
+
+
+def test_decode_wait_limit_returns_and_recovers():
+    """The batch-1 decode kernel waits (bounded) on its weight copies.  With the
+    cap at one try a wait may or may not run out, depending on whether the
+    copy has landed; either way the call returns, a timeout is latched as
+    BITNET_ERR_TIMEOUT, and the next call is exact."""
+    tt = torch()
+    if not tt.cuda.is_available():
+        pytest.skip("no CUDA device")
+    b = lib()
+    rows, K = 13824, 2560
+    t = syn.ternary_uniform(81, rows, K)
+    sc = syn.positive_scales(82, rows, K // 128, per_tensor=True)
+    x = syn.activations(83, 1, K)
+    w, _ = device_weight(t, sc)
+    xd = tt.from_numpy(x.reshape(-1).copy()).cuda()
+    y = tt.empty(rows, dtype=tt.float32, device="cuda")
+    assert b.bitnet_get_device_error() == b.BITNET_OK
+    b.bitnet_set_wait_limit(1)
+    try:
+        for _ in range(4):
+            b.bitnet_w2a8_linear(w, xd, 1, y)
+        st = b.bitnet_get_device_error()
+    finally:
+        b.bitnet_set_wait_limit(0)
+    assert st in (b.BITNET_OK, b.BITNET_ERR_TIMEOUT)
+    assert b.bitnet_get_device_error() == b.BITNET_OK
+    b.bitnet_w2a8_linear(w, xd, 1, y)
+    assert b.bitnet_get_device_error() == b.BITNET_OK
+    rq, rs, _ = oracle.quant_act(x)
+    np.testing.assert_array_equal(to_np(y).reshape(1, rows), oracle.linear(oracle.pack_i2s(t), sc, K, rq, rs))
