@@ -575,7 +575,8 @@ def cpu_baseline(seconds=12.0):
 
 def run_case(args):
     """One kernel on one shape, for profiling: `--case gemv` runs
-    bitnet_w2a8_gemv over `--copies` distinct weights (so the weights exceed
+    bitnet_w2a8_gemv and `--case linear` bitnet_w2a8_linear (activation
+    quantisation fused) over `--copies` distinct weights (so the weights exceed
     L2), `--case gemm` runs bitnet_w2a8_gemm on one weight; `--reps` passes,
     plain launches (no graph).  Prints one JSON line with the median time."""
     import torch
@@ -586,15 +587,20 @@ def run_case(args):
     torch.cuda.set_device(dev)
     o, k = args.rows, args.cols
     seed = 0xB17E7 ^ 0x5A5A
-    copies = args.copies if args.case == "gemv" else 1
+    vec = args.case in ("gemv", "linear")
+    copies = args.copies if vec else 1
     ws = build_weights(b, torch, dev, copies, [("w", o, k)], seed)
-    T = args.batch if args.case == "gemv" else args.tokens
+    T = args.batch if vec else args.tokens
     x = torch.randn(T * k, dtype=torch.float32, device=dev)
     q = torch.empty(T * k, dtype=torch.int8, device=dev)
     s = torch.empty(T, dtype=torch.float32, device=dev)
     y = torch.empty(T * o, dtype=torch.float32, device=dev)
     b.bitnet_quant_act(x, T, k, q, s)
-    call = b.bitnet_w2a8_gemv if args.case == "gemv" else b.bitnet_w2a8_gemm
+    if args.case == "linear":
+        def call(w, q_, s_, T_, y_):
+            b.bitnet_w2a8_linear(w, x, T_, y_)
+    else:
+        call = b.bitnet_w2a8_gemv if args.case == "gemv" else b.bitnet_w2a8_gemm
     times = []
     for _ in range(args.reps):
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -607,8 +613,9 @@ def run_case(args):
     assert b.bitnet_get_device_error() == b.BITNET_OK
     med = sorted(times)[len(times) // 2]
     out = {"case": args.case, "out": o, "K": k, "T": T, "copies": copies, "us_per_launch": round(med, 3)}
-    if args.case == "gemv":
-        out["GB/s"] = round(gemv_bytes(o, k, T) / (med * 1e-6) / 1e9, 1)
+    if vec:
+        nbytes = gemv_bytes(o, k, T) if args.case == "gemv" else linear_bytes(o, k, T)
+        out["GB/s"] = round(nbytes / (med * 1e-6) / 1e9, 1)
     else:
         out["TOPS"] = round(2.0 * T * o * k / (med * 1e-6) / 1e12, 1)
     print(json.dumps(out), flush=True)
@@ -623,7 +630,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--case", choices=["gemv", "gemm"], help="profile one kernel on one shape")
+    ap.add_argument("--case", choices=["gemv", "linear", "gemm"], help="profile one kernel on one shape")
     ap.add_argument("--rows", type=int, default=13824)
     ap.add_argument("--cols", type=int, default=2560)
     ap.add_argument("--batch", type=int, default=1)

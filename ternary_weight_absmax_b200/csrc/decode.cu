@@ -66,8 +66,8 @@ struct DecArgs {
     int nb;
     int tiles_lo;  // every CTA owns tiles_lo or tiles_lo + 1 row tiles
     int extra;     // the first `extra` CTAs own tiles_lo + 1
-    int wcap;      // tiles of shared memory per warp: kChunk * (copies in flight)
-    uint32_t off_q, off_acc, off_rsc, off_red, off_bar;
+    int wcap;      // tiles of shared memory per warp: kChunk * (copies in flight), a power of two
+    uint32_t off_q, off_acc, off_rsc, off_rsd, off_red, off_bar;
 };
 
 // Shared-memory word of activation word m (bytes 4m .. 4m+3 of q): lane-part t
@@ -78,12 +78,24 @@ __device__ __forceinline__ int perm_word(int m) {
     return (m & ~31) | ((w & 3) << 3) | ((w >> 3) << 1) | ((w >> 2) & 1);
 }
 
-// Lane 0 waits on the mbarrier phase (bounded), the warp gets the verdict.
-__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, uint32_t limit) {
-    int ok = 0;
-    if ((threadIdx.x & 31) == 0) ok = ptx::mbar_wait(bar, parity, limit, nullptr) ? 1 : 0;
-    ok = __shfl_sync(0xffffffffu, ok, 0);
-    return ok != 0;
+// Exact int32 -> fp64 with one integer op and one fp64 add: the bits
+// 0x43300000:(v ^ 0x80000000) encode 2^52 + 2^31 + v.
+__device__ __forceinline__ double int_to_double(int v) {
+    return __hiloint2double(0x43300000, (int)((unsigned)v ^ 0x80000000u)) - 4503601774854144.0;
+}
+
+// The activation quantiser's rounding, clamp(rint(v), -127, 127) with ties
+// to even, for |v| < 2^22 (here |v| <= 127 * (1 + 2^-23)): adding 1.5 * 2^23
+// leaves rint(v) in the low mantissa bits.  NaN gives 0, as __float2int_rn.
+__device__ __forceinline__ uint32_t quant1(float x, float s) {
+    const float v = __fmul_rn(x, s);
+    int q = __float_as_int(__fadd_rn(v, 12582912.0f)) - 0x4B400000;
+    q = q > 127 ? 127 : (q < -127 ? -127 : q);
+    return v == v ? (uint32_t)(q & 0xff) : 0u;
+}
+
+__device__ __forceinline__ uint32_t quant4_fast(float4 v, float s) {
+    return quant1(v.x, s) | (quant1(v.y, s) << 8) | (quant1(v.z, s) << 16) | (quant1(v.w, s) << 24);
 }
 
 template <bool FUSED, int NX>
@@ -97,12 +109,14 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const DecArgs a)
     const int n = nr * a.nb;
     const int i0 = (int)(((int64_t)warp * n) / kWarps);
     const int nit = (int)(((int64_t)(warp + 1) * n) / kWarps) - i0;
-    const int nslots = a.wcap / kChunk;
+    const int wcap = a.wcap;  // a power of two, kChunk .. kChunk * kMaxSlots
+    const int nslots = wcap / kChunk;
     const int nchunks = (nit + kChunk - 1) / kChunk;
-    unsigned char *wsm = smem + (size_t)warp * a.wcap * kTile;
+    unsigned char *wsm = smem + (size_t)warp * wcap * kTile;
     uint32_t *qw = reinterpret_cast<uint32_t *>(smem + a.off_q);
     int *acc = reinterpret_cast<int *>(smem + a.off_acc);
     float *rsc = reinterpret_cast<float *>(smem + a.off_rsc);
+    double *rsd = reinterpret_cast<double *>(smem + a.off_rsd);
     unsigned *wmax = reinterpret_cast<unsigned *>(smem + a.off_red);
     int *wqs = reinterpret_cast<int *>(smem + a.off_red + 64);
     const uint32_t bars = ptx::smem_u32(smem + a.off_bar) + 8u * (warp * kMaxSlots);
@@ -115,17 +129,18 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const DecArgs a)
     // ---- before the wait: nothing here depends on the previous kernel.
     const uint64_t pol = ptx::policy_evict_first();
     auto issue = [&](int k) {  // lane 0: chunk k of this warp's tiles into its slot
-        const int s = k % nslots;
+        const int s = k & (nslots - 1);
         const uint32_t bytes = (uint32_t)min(kChunk, nit - k * kChunk) * kTile;
         ptx::mbar_arrive_expect_tx(bars + 8u * s, bytes);
         ptx::bulk_g2s(ptx::smem_u32(wsm + s * kChunk * kTile), src + (size_t)k * kChunk * kTile, bytes,
                       bars + 8u * s, pol);
     };
+    const int npre = nchunks < nslots ? nchunks : nslots;
     if (lane == 0) {
         for (int s = 0; s < nslots; s++) ptx::mbar_init(bars + 8u * s, 1);
         if (warp == 0) ptx::mbar_init(rbar, 1);
         ptx::fence_mbar_init();
-        for (int k = 0; k < nchunks && k < nslots; k++) issue(k);
+        for (int k = 0; k < npre; k++) issue(k);
         if (warp == 0) {
             const uint32_t bytes = (uint32_t)nr * kTileRows * sizeof(float);
             ptx::mbar_arrive_expect_tx(rbar, bytes);
@@ -133,12 +148,36 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const DecArgs a)
         }
     }
     for (int i = tid; i < nr * kTileRows; i += kThreads) acc[i] = 0;
+    // Index state of the product loop, set up here, off the critical path.
+    const int r = i0 / a.nb;
+    int j = i0 - r * a.nb;
+    int *accp = acc + r * kTileRows + g;  // rows g and g + 8 of the current tile
+    const uint4 *qrow = reinterpret_cast<const uint4 *>(qw + t * 8);  // block 0, this lane's part
+    const uint4 *qp = qrow + j * 8;
+    const uint4 *wl = reinterpret_cast<const uint4 *>(wsm) + lane;
+    // Wait for the copies issued above while the previous kernel still runs
+    // (a wait is cheap here and costly after griddepcontrol.wait).
+    bool ok = true;
+    for (int k = 0; k < npre && ok; k++) {
+        int got = 0;
+        if (lane == 0) got = ptx::mbar_wait_sleep(bars + 8u * k, 0u, limit, nullptr, 64) ? 1 : 0;
+        ok = __shfl_sync(0xffffffffu, got, 0) != 0;
+    }
+    if (warp == 0) {
+        int got = 0;
+        if (lane == 0) got = ptx::mbar_wait_sleep(rbar, 0u, limit, nullptr, 64) ? 1 : 0;
+        if (!__shfl_sync(0xffffffffu, got, 0)) ok = false;
+        // Row scales to fp64 now, so the epilogue does no conversion of them.
+        if (ok)
+            for (int i = lane; i < nr * kTileRows; i += 32) rsd[i] = (double)rsc[i];
+    }
 
     asm volatile("griddepcontrol.wait;" ::: "memory");  // x (or q, s) ready; y free
 
     // ---- activations: s, q (permuted) in shared memory, sum(q).
     const int K4 = a.K >> 2;
     float s;
+    double sd;
     int qsum = 0;
     if constexpr (FUSED) {
         const float4 *x4 = reinterpret_cast<const float4 *>(a.x);
@@ -162,13 +201,14 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const DecArgs a)
         }
         const float amax = __uint_as_float(mm);
         s = __fdiv_rn(127.0f, amax > kEps ? amax : kEps);
+        sd = (double)s;
         if (c == 0 && tid == 0 && a.s_out) a.s_out[0] = s;
         uint32_t *qo = (c == 0 && a.q_out) ? reinterpret_cast<uint32_t *>(a.q_out) : nullptr;
 #pragma unroll
         for (int u = 0; u < NX; u++) {
             const int i = tid + u * kThreads;
             if (i < K4) {
-                const uint32_t w = quant4(xv[u], s);
+                const uint32_t w = quant4_fast(xv[u], s);
                 qw[perm_word(i)] = w;
                 qsum = dp4a_ss((int)w, 0x01010101, qsum);
                 if (qo) qo[i] = w;
@@ -176,6 +216,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const DecArgs a)
         }
     } else {
         s = *a.s;
+        sd = (double)s;
         const uint32_t *q4 = reinterpret_cast<const uint32_t *>(a.q);
         for (int i = tid; i < K4; i += kThreads) {
             const uint32_t w = q4[i];
@@ -186,14 +227,17 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const DecArgs a)
     qsum = __reduce_add_sync(0xffffffffu, qsum);
     if (lane == 0) wqs[warp] = qsum;
     __syncthreads();
+    int tot = 0;  // sum(q) over the row
+#pragma unroll
+    for (int w = 0; w < kWarps / 4; w++) {
+        const int4 v = reinterpret_cast<const int4 *>(wqs)[w];
+        tot += v.x + v.y + v.z + v.w;
+    }
 
-    // ---- products.  Items of this warp: i0 .. i0 + nit - 1, tile r = i / nb,
-    // block j = i % nb; the four group sums of rows g and g + 8 are held until
-    // the tile changes.
+    // ---- products.  Items of this warp: i0 .. i0 + nit - 1 (tile r = i / nb,
+    // block j = i % nb), item `it` in shared-memory slot it % wcap; the four
+    // group sums of rows g and g + 8 are held until the tile changes.
     int aA[4] = {0, 0, 0, 0}, aB[4] = {0, 0, 0, 0};
-    const int r = i0 / a.nb;
-    int j = i0 - r * a.nb;
-    int *accp = acc + r * kTileRows + g;  // rows g and g + 8 of the current tile
     auto flush = [&]() {
         const int pA = tig_reduce(combine4(aA));
         const int pB = tig_reduce(combine4(aB));
@@ -204,78 +248,91 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const DecArgs a)
 #pragma unroll
         for (int k = 0; k < 4; k++) aA[k] = aB[k] = 0;
     };
-    int k = 0;
-    bool ok = true;
-    for (; k < nchunks; k++) {
-        const int slot = k % nslots;
-        if (!warp_wait(bars + 8u * slot, (uint32_t)(k / nslots) & 1u, limit)) {
-            ok = false;
-            break;
+    // The products of one item: tile word w (lane's 16 bytes), activation
+    // words at qv (qa0 qb0 qa1 qb1 | qa2 qb2 qa3 qb3).
+    auto item = [&](const uint4 w, const uint4 *qv) {
+        const uint4 q0 = qv[0], q1 = qv[1];
+        const int qa[4] = {(int)q0.x, (int)q0.z, (int)q1.x, (int)q1.z};
+        const int qb[4] = {(int)q0.y, (int)q0.w, (int)q1.y, (int)q1.w};
+#pragma unroll
+        for (int gg = 0; gg < 4; gg++) {
+            const uint32_t mk = 0xC0C0C0C0u >> (2 * gg);
+            aA[gg] = dp4a_us(w.x & mk, qa[gg], aA[gg]);
+            aA[gg] = dp4a_us(w.z & mk, qb[gg], aA[gg]);
+            aB[gg] = dp4a_us(w.y & mk, qa[gg], aB[gg]);
+            aB[gg] = dp4a_us(w.w & mk, qb[gg], aB[gg]);
         }
-        const uint4 *cw = reinterpret_cast<const uint4 *>(wsm + slot * kChunk * kTile) + lane;
-        const int m = min(kChunk, nit - k * kChunk);
-#pragma unroll
-        for (int e = 0; e < kChunk; e++) {
-            if (e >= m) break;
-            const uint4 w = cw[e * 32];
-            const uint4 *qp = reinterpret_cast<const uint4 *>(qw + j * 32 + t * 8);
-#pragma unroll
-            for (int h = 0; h < 2; h++) {
-                const uint4 qv = qp[h];  // qa, qb of groups 2h and 2h + 1
-#pragma unroll
-                for (int f = 0; f < 2; f++) {
-                    const int gg = 2 * h + f;
-                    const int qa = (int)(f ? qv.z : qv.x), qb = (int)(f ? qv.w : qv.y);
-                    const uint32_t mk = 0xC0C0C0C0u >> (2 * gg);
-                    aA[gg] = dp4a_us(w.x & mk, qa, aA[gg]);
-                    aA[gg] = dp4a_us(w.z & mk, qb, aA[gg]);
-                    aB[gg] = dp4a_us(w.y & mk, qa, aB[gg]);
-                    aB[gg] = dp4a_us(w.w & mk, qb, aB[gg]);
+    };
+    int it = 0;
+    if (nit <= wcap) {
+        // Every tile of the warp is already in shared memory: runs of items
+        // within one row tile, one flush per run.
+        while (it < nit && ok) {
+            const int run = min(nit - it, a.nb - j);
+            const uint4 *wv = wl + it * 32;
+#pragma unroll 2
+            for (int e = 0; e < run; e++) item(wv[e * 32], qp + e * 8);
+            it += run;
+            j += run;
+            qp += run * 8;
+            if (j == a.nb) {
+                flush();
+                accp += kTileRows;
+                j = 0;
+                qp = qrow;
+            }
+        }
+    } else {
+        // Streaming: item `it` sits in slot it % wcap; chunks from nslots on
+        // are waited for here and refilled as their slots free up.
+        for (; it < nit && ok; it++) {
+            if (it >= wcap && (it & (kChunk - 1)) == 0) {
+                const int k = it / kChunk;
+                int got = 0;
+                if (lane == 0)
+                    got = ptx::mbar_wait(bars + 8u * (k & (nslots - 1)), (uint32_t)(k / nslots) & 1u, limit,
+                                         nullptr) ? 1 : 0;
+                if (!__shfl_sync(0xffffffffu, got, 0)) {
+                    ok = false;
+                    break;
                 }
             }
+            item(wl[(it & (wcap - 1)) * 32], qp);
+            qp += 8;
             if (++j == a.nb) {
                 flush();
                 accp += kTileRows;
                 j = 0;
+                qp = qrow;
             }
-        }
-        if (k + nslots < nchunks) {
-            __syncwarp();  // every lane has read the slot
-            if (lane == 0) {
-                ptx::fence_proxy_async_smem();
-                issue(k + nslots);
+            if ((it & (kChunk - 1)) == kChunk - 1 && it / kChunk + nslots < nchunks) {
+                __syncwarp();  // every lane has read the chunk's slot
+                if (lane == 0) {
+                    ptx::fence_proxy_async_smem();
+                    issue(it / kChunk + nslots);
+                }
             }
         }
     }
     if (!ok) {
-        // Timed out: record it, then wait out this warp's copies still in flight.
+        // Timed out: record it, then wait out this warp's copies still in flight
+        // (chunks it / kChunk .. the last one issued).
         if (lane == 0) {
             atomicOr(a.err, kErrTimeout);
-            for (int kk = k; kk < nchunks && kk < k + nslots; kk++)
-                ptx::mbar_wait(bars + 8u * (kk % nslots), (uint32_t)(kk / nslots) & 1u, kDrainLimit, nullptr);
+            const int k0 = it / kChunk;
+            for (int k = k0; k < nchunks && k < k0 + nslots; k++)
+                ptx::mbar_wait(bars + 8u * (k & (nslots - 1)), (uint32_t)(k / nslots) & 1u, kDrainLimit, nullptr);
+            if (warp == 0) ptx::mbar_wait(rbar, 0u, kDrainLimit, nullptr);
         }
         __syncwarp();
     }
     if (j != 0) flush();  // items since the last tile change (none if j == 0)
-    if (warp == 0 && !warp_wait(rbar, 0u, limit)) {
-        if (lane == 0) {
-            atomicOr(a.err, kErrTimeout);
-            ptx::mbar_wait(rbar, 0u, kDrainLimit, nullptr);
-        }
-        __syncwarp();
-    }
     __syncthreads();
 
     // ---- epilogue: y = rowscale * (sum c*q - sum q) / s, fp64, one rounding.
-    int tot = 0;
-#pragma unroll
-    for (int w = 0; w < kWarps / 4; w++) {
-        const int4 v = reinterpret_cast<const int4 *>(wqs)[w];
-        tot += v.x + v.y + v.z + v.w;
-    }
     for (int i = tid; i < nr * kTileRows; i += kThreads) {
         const int64_t o = r0 * kTileRows + i;
-        if (o < a.rows) a.y[o] = (float)((double)rsc[i] * (double)(acc[i] - tot) / (double)s);
+        if (o < a.rows) a.y[o] = __double2float_rn(rsd[i] * int_to_double(acc[i] - tot) / sd);
     }
 }
 
@@ -296,14 +353,14 @@ bool plan(const Layout &L, bool fused, Plan *p) {
     if (fused && nx > 8) return false;
     const int64_t lo = L.ntr / grid, hi = lo + (L.ntr % grid ? 1 : 0);
     const int64_t per_warp = (hi * L.nb + kWarps - 1) / kWarps;
-    int wcap = (int)(per_warp < kChunk * kMaxSlots ? per_warp : kChunk * kMaxSlots);
-    wcap = (wcap + kChunk - 1) / kChunk * kChunk;
-    if (wcap < kChunk) wcap = kChunk;
+    int wcap = kChunk;  // power of two >= the tiles of a warp, at most kChunk * kMaxSlots
+    while (wcap < per_warp && wcap < kChunk * kMaxSlots) wcap *= 2;
     DecArgs &a = p->a;
     a.off_q = (uint32_t)(kWarps * wcap * kTile);
     a.off_acc = (uint32_t)align_up(a.off_q + (size_t)K, 16);
     a.off_rsc = a.off_acc + (uint32_t)(hi * kTileRows * sizeof(int));
-    a.off_red = a.off_rsc + (uint32_t)(hi * kTileRows * sizeof(float));
+    a.off_rsd = (uint32_t)align_up(a.off_rsc + (size_t)hi * kTileRows * sizeof(float), 16);
+    a.off_red = a.off_rsd + (uint32_t)(hi * kTileRows * sizeof(double));
     a.off_bar = a.off_red + 128;
     const size_t smem = a.off_bar + 8 * (kWarps * kMaxSlots + 1);
     if (smem > 100 * 1024) return false;  // two CTAs per SM
