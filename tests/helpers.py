@@ -66,3 +66,17 @@ def assert_close(y, ref, what=""):
         bad = np.argwhere(~ok)[:5]
         raise AssertionError(f"{what}: {int((~ok).sum())} of {ok.size} outside 1e-6*|ref|+1e-6; "
                              f"first {bad.tolist()} y={np.asarray(y)[tuple(bad.T)]} ref={np.asarray(ref)[tuple(bad.T)]}")
+
+
+def assert_decode_close(y, ref, what=""):
+    """Outputs of the batch-1 decode kernel (uniform rows), whose epilogue runs
+    in fp32: rowscale * sum * (1/s) with three roundings, so within 3 * 2^-24
+    of the exact value and within 4e-7 of the fp64 oracle (tighter than the
+    1e-6*|ref| + 1e-6 bar, which it must also meet).  Zero sums give zero."""
+    assert_close(y, ref, what)
+    y = np.asarray(y, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    zero = ref == 0.0
+    assert np.all(y[zero] == 0.0), f"{what}: nonzero output where the oracle gives 0"
+    rel = np.abs(y[~zero] - ref[~zero]) / np.abs(ref[~zero])
+    assert rel.size == 0 or rel.max() <= 4e-7, f"{what}: relative error {rel.max():.3e} above 4e-7"

@@ -6,7 +6,7 @@ import numpy as np
 import pytest
 
 import oracle
-from helpers import assert_close, device_weight, gpu_quant, lib, to_np, torch
+from helpers import assert_close, assert_decode_close, device_weight, gpu_quant, lib, to_np, torch
 import synthetic as syn
 
 pytestmark = pytest.mark.gpu
@@ -43,7 +43,7 @@ def test_decode_wait_limit_returns_and_recovers():
     """The batch-1 decode kernel waits (bounded) on its weight copies.  With the
     cap at one try a wait may or may not run out, depending on whether the
     copy has landed; either way the call returns, a timeout is latched as
-    BITNET_ERR_TIMEOUT, and the next call is exact."""
+    BITNET_ERR_TIMEOUT, and the next call is correct."""
     tt = torch()
     if not tt.cuda.is_available():
         pytest.skip("no CUDA device")
@@ -68,4 +68,4 @@ def test_decode_wait_limit_returns_and_recovers():
     b.bitnet_w2a8_linear(w, xd, 1, y)
     assert b.bitnet_get_device_error() == b.BITNET_OK
     rq, rs, _ = oracle.quant_act(x)
-    np.testing.assert_array_equal(to_np(y).reshape(1, rows), oracle.linear(oracle.pack_i2s(t), sc, K, rq, rs))
+    assert_decode_close(to_np(y).reshape(1, rows), oracle.linear(oracle.pack_i2s(t), sc, K, rq, rs), "after limit")
