@@ -360,14 +360,17 @@ def run_ours(args, rank, world, dev):
     e2e_value, _ = aggregate([e2e_ms] * world, [per_rank_bytes] * world)
 
     peaks = read_peaks()
-    gemv_launch_us = gemv_ms_max * 1e3 / gemv_launches
-    gemv_bytes_per_launch = gbytes / gemv_launches
-    achieved = gemv_bytes_per_launch / (gemv_launch_us * 1e-6) / 1e9
-    roofline = {"kernel": "gemv_b1_kernel (bitnet_w2a8_gemv, B=1)", "bound": "hbm",
+    # Dominant kernel: the batch-1 decode kernel behind bitnet_w2a8_linear, one
+    # launch per linear of the step; its average launch time is the step time
+    # (CUDA events on the launch stream, timed region above) over the launches.
+    launch_us = step_ms * 1e3 / launches_per_step
+    bytes_per_launch = per_rank_bytes / launches_per_step
+    achieved = bytes_per_launch / (launch_us * 1e-6) / 1e9
+    roofline = {"kernel": "decode_b1_kernel (bitnet_w2a8_linear, batch 1, uniform rows)", "bound": "hbm",
                 "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": round(achieved / peaks["hbm_gbs"], 4), "peak_source": peaks["source"],
-                "traffic": read_traffic(), "bytes_per_launch": gemv_bytes_per_launch,
-                "launch_us": round(gemv_launch_us, 3)}
+                "traffic": read_traffic(), "bytes_per_launch": round(bytes_per_launch, 1),
+                "launch_us": round(launch_us, 3)}
 
     out = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
@@ -467,8 +470,9 @@ def read_peaks():
 
 
 def read_traffic():
-    """DRAM bytes per GEMV launch from the committed ncu summary, if present."""
-    p = os.path.join(ROOT, "profiles", "gemv_traffic.json")
+    """DRAM bytes per decode-kernel launch (mean over the step's four shapes)
+    from the committed ncu summary, if present."""
+    p = os.path.join(ROOT, "profiles", "decode_traffic.json")
     try:
         with open(p) as f:
             return json.load(f).get("bytes_per_launch")
