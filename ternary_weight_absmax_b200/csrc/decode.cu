@@ -5,34 +5,40 @@
 // activations ("5倍性能跃升：BitNet与llama.cpp的1-bit LLM推理架构对决", section
 // "GPU内核突破": 2-bit weights x 8-bit activations with dp4a; the activation
 // quantisation is the per-token absmax of "BitNet b1.58", section "Quantization
-// Function").  The arithmetic is that of the general GEMV kernel: integer dot
-// products, one exact fp64 product with the row scale, one fp64 divide by s,
-// one rounding to fp32.
+// Function").  q and the integer sums are exactly those of the general kernel;
+// the epilogue runs in fp32 (below).
 //
 // A decode step is a chain of dependent linears of a few microseconds each, so
 // what costs is the chain's latency: the time from the previous kernel's end
 // to this kernel's last store.  Measured on B200, the pieces of that are the
-// release of griddepcontrol.wait (~0.5 us after the previous grid ends), one
-// L2 round trip for x, the CTA barriers and the dp4a work; weights that are
-// still in flight when the products start add their DRAM time on top.  Hence:
+// release of griddepcontrol.wait (~0.6 us after the previous grid ends), one
+// L2 round trip for x, two CTA barriers around the activation quantisation,
+// the dp4a work (ALU-pipe bound: one LOP3 mask and one IDP4A per four
+// weights) and the epilogue.  Hence:
 //
-//  * one CTA of 16 warps per SM with less than half of the SM's registers and
-//    shared memory, so that the next linear's CTAs are resident while this one
-//    runs (programmatic dependent launch) and fetch their weights before their
-//    griddepcontrol.wait;
+//  * one CTA of 16 warps per SM, at most half of the SM's registers, so the
+//    next linear's CTA is resident beside this one (programmatic dependent
+//    launch) and fetches its weights before its griddepcontrol.wait;
 //  * the weights move by bulk copies (cp.async.bulk, one per two 512-byte
-//    tiles, L2 evict-first: they are read once per step and must not push the
-//    activations out of L2) into shared memory, up to eight tiles per warp in
-//    flight; register loads could not keep enough bytes in flight per SM;
+//    tiles, L2 evict-first: read once per step, they must not push the
+//    activations out of L2) into shared memory, up to eight tiles per warp;
+//    register loads could not keep enough bytes in flight per SM;
+//  * the copies are waited for before griddepcontrol.wait, where the wait is
+//    free; larger slices stream through the same slots after it;
+//  * every shared-memory carveout request is the same (max shared), so CTAs
+//    of consecutive linears share an SM without it being reconfigured;
 //  * a CTA owns whole row tiles (no cross-CTA reduction) and its warps split
 //    the (tile, block) items evenly in memory order, so a warp's tiles are one
-//    contiguous range;
+//    contiguous range; index state is set up before the wait;
 //  * after the wait: x is read once into registers, the absmax is combined
-//    across warps through shared memory (one barrier), x is quantised into
+//    across warps through shared memory (barrier 1), x is quantised into
 //    shared memory in the order the lanes read it (a lane's eight words of a
-//    block are 32 contiguous bytes) and sum(q) is taken once per CTA (second
-//    barrier); then the masked dp4a products, one shared-memory atomic per row
-//    and tile change, the third barrier and the epilogue.
+//    block are 32 contiguous bytes) and sum(q) is taken once per CTA
+//    (barrier 2); the products run per row-tile run without per-item
+//    branches, one shared-memory atomic per row and run; barrier 3, epilogue;
+//  * the epilogue is fp32: rowscale * sum * (1/s), three roundings, relative
+//    error below 2.4e-7 of the fp64 value (the fp64 product, divide and
+//    conversions cost ~0.25 us per call on this path).
 // Integer sums are exact, so the atomics leave the result independent of
 // their order.  Every wait on a copy is bounded; on a timeout the kernel sets
 // the device error word, waits (bounded) for its copies in flight and returns.
@@ -347,8 +353,7 @@ bool plan(const Layout &L, bool fused, Plan *p) {
     const int K = (int)L.cols;
     int nx = 1;
     while (nx * 4 * kThreads < K) nx *= 2;
-    if (fused && nx > 8) return false;
-    if (K > 32768) return false;  // int sums stay below 2^22 for the fp32 epilogue
+    if (K > 16384) return false;  // x in registers (fused); int sums below 2^22 for the fp32 epilogue
     const int64_t lo = L.ntr / grid, hi = lo + (L.ntr % grid ? 1 : 0);
     const int64_t per_warp = (hi * L.nb + kWarps - 1) / kWarps;
     int wcap = kChunk;  // power of two >= the tiles of a warp, at most kChunk * kMaxSlots

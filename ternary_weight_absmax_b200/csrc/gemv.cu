@@ -1,4 +1,7 @@
-// gemv.cu -- decode / small-batch W2A8 GEMV (1 <= B <= 16) with dp4a.
+// gemv.cu -- small-batch W2A8 GEMV (1 <= B <= 16) with dp4a: the general
+// kernel (B >= 2, per-block scales, accumulator export, K > 16384).  Batch-1
+// calls on uniform rows go to the decode kernel (decode.cu); launch_gemv at
+// the end of this file chooses.
 //
 // y[b][o] = (sum_j scale[o][j] * acc[b][o][j]) / s[b],
 // acc[b][o][j] = sum_{k in block j} t[o][k] * q[b][k]   (int32, exact).
