@@ -90,18 +90,19 @@ __device__ __forceinline__ float int_to_float(int v) {
     return __fsub_rn(__int_as_float(0x4B400000 + v), 12582912.0f);
 }
 
-// The activation quantiser's rounding, clamp(rint(v), -127, 127) with ties
-// to even, for |v| < 2^22 (here |v| <= 127 * (1 + 2^-23)): adding 1.5 * 2^23
-// leaves rint(v) in the low mantissa bits.  NaN gives 0, as __float2int_rn.
-__device__ __forceinline__ uint32_t quant1(float x, float s) {
-    const float v = __fmul_rn(x, s);
-    int q = __float_as_int(__fadd_rn(v, 12582912.0f)) - 0x4B400000;
-    q = q > 127 ? 127 : (q < -127 ? -127 : q);
-    return v == v ? (uint32_t)(q & 0xff) : 0u;
-}
-
+// The activation quantiser's q = rint(x * s) (one fp32 multiply, ties to
+// even) for four activations of a row with |x| <= absmax: then
+// |x * s| <= 127 * (1 + 2^-24)^2 < 127.5, so q lies in [-127, 127] and the
+// clamp never acts for finite x.  Adding 1.5 * 2^23 (round-to-nearest-even)
+// leaves rint(v) in the low mantissa bits, and the low byte of those bits is q
+// as an int8; three byte permutes pack the four bytes.  (NaN or Inf in x give
+// unspecified bytes here.)
 __device__ __forceinline__ uint32_t quant4_fast(float4 v, float s) {
-    return quant1(v.x, s) | (quant1(v.y, s) << 8) | (quant1(v.z, s) << 16) | (quant1(v.w, s) << 24);
+    const uint32_t b0 = __float_as_uint(__fadd_rn(__fmul_rn(v.x, s), 12582912.0f));
+    const uint32_t b1 = __float_as_uint(__fadd_rn(__fmul_rn(v.y, s), 12582912.0f));
+    const uint32_t b2 = __float_as_uint(__fadd_rn(__fmul_rn(v.z, s), 12582912.0f));
+    const uint32_t b3 = __float_as_uint(__fadd_rn(__fmul_rn(v.w, s), 12582912.0f));
+    return __byte_perm(__byte_perm(b0, b1, 0x0040), __byte_perm(b2, b3, 0x0040), 0x5410);
 }
 
 template <bool FUSED, int NX>
@@ -122,8 +123,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const DecArgs a)
     uint32_t *qw = reinterpret_cast<uint32_t *>(smem + a.off_q);
     int *acc = reinterpret_cast<int *>(smem + a.off_acc);
     float *rsc = reinterpret_cast<float *>(smem + a.off_rsc);
-    unsigned *wmax = reinterpret_cast<unsigned *>(smem + a.off_red);
-    int *wqs = reinterpret_cast<int *>(smem + a.off_red + 64);
+    unsigned *amax_w = reinterpret_cast<unsigned *>(smem + a.off_red);  // absmax bits (atomic max)
+    int *qsum_w = reinterpret_cast<int *>(smem + a.off_red + 4);          // sum(q) (atomic add)
     const uint32_t bars = ptx::smem_u32(smem + a.off_bar) + 8u * (warp * kMaxSlots);
     const uint32_t rbar = ptx::smem_u32(smem + a.off_bar) + 8u * (kWarps * kMaxSlots);
     const unsigned char *src = a.tiles + (size_t)(r0 * a.nb + i0) * kTile;
@@ -153,6 +154,10 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const DecArgs a)
         }
     }
     for (int i = tid; i < nr * kTileRows; i += kThreads) acc[i] = 0;
+    if (tid == 0) {
+        *amax_w = 0u;
+        *qsum_w = 0;
+    }
     // Index state of the product loop, set up here, off the critical path.
     const int r = i0 / a.nb;
     int j = i0 - r * a.nb;
@@ -174,6 +179,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const DecArgs a)
         if (!__shfl_sync(0xffffffffu, got, 0)) ok = false;
     }
 
+    __syncthreads();  // acc and the two reduction words are zero for every warp
     asm volatile("griddepcontrol.wait;" ::: "memory");  // x (or q, s) ready; y free
 
     // ---- activations: s, q (permuted) in shared memory, sum(q).
@@ -192,15 +198,9 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const DecArgs a)
         }
         // m >= 0 and not NaN (fmaxf drops NaN): its bit pattern orders like its value.
         const unsigned mu = __reduce_max_sync(0xffffffffu, __float_as_uint(m));
-        if (lane == 0) wmax[warp] = mu;
+        if (lane == 0) atomicMax(amax_w, mu);
         __syncthreads();
-        unsigned mm = 0u;
-#pragma unroll
-        for (int k = 0; k < kWarps / 4; k++) {
-            const uint4 v = reinterpret_cast<const uint4 *>(wmax)[k];
-            mm = max(mm, max(max(v.x, v.y), max(v.z, v.w)));
-        }
-        const float amax = __uint_as_float(mm);
+        const float amax = __uint_as_float(*amax_w);
         s = __fdiv_rn(127.0f, amax > kEps ? amax : kEps);
         inv_s = __frcp_rn(s);
         if (c == 0 && tid == 0 && a.s_out) a.s_out[0] = s;
@@ -226,14 +226,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const DecArgs a)
         }
     }
     qsum = __reduce_add_sync(0xffffffffu, qsum);
-    if (lane == 0) wqs[warp] = qsum;
+    if (lane == 0) atomicAdd(qsum_w, qsum);
     __syncthreads();
-    int tot = 0;  // sum(q) over the row
-#pragma unroll
-    for (int w = 0; w < kWarps / 4; w++) {
-        const int4 v = reinterpret_cast<const int4 *>(wqs)[w];
-        tot += v.x + v.y + v.z + v.w;
-    }
 
     // ---- products.  Items of this warp: i0 .. i0 + nit - 1 (tile r = i / nb,
     // block j = i % nb), item `it` in shared-memory slot it % wcap; the four
@@ -330,6 +324,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const DecArgs a)
     if (j != 0) flush();  // items since the last tile change (none if j == 0)
     __syncthreads();
 
+    const int tot = *qsum_w;  // sum(q) over the row
     // ---- epilogue: y = rowscale * (sum c*q - sum q) * (1/s) in fp32: three
     // roundings, relative error below 2e-7 (the int sum is exact in fp32,
     // |sum| <= 127 * K < 2^22).  The general kernel keeps the fp64 epilogue.
