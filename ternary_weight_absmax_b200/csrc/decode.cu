@@ -125,6 +125,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const DecArgs a)
     float *rsc = reinterpret_cast<float *>(smem + a.off_rsc);
     unsigned *amax_w = reinterpret_cast<unsigned *>(smem + a.off_red);  // absmax bits (atomic max)
     int *qsum_w = reinterpret_cast<int *>(smem + a.off_red + 4);          // sum(q) (atomic add)
+    int *bad_w = reinterpret_cast<int *>(smem + a.off_red + 8);           // a copy wait ran out
     const uint32_t bars = ptx::smem_u32(smem + a.off_bar) + 8u * (warp * kMaxSlots);
     const uint32_t rbar = ptx::smem_u32(smem + a.off_bar) + 8u * (kWarps * kMaxSlots);
     const unsigned char *src = a.tiles + (size_t)(r0 * a.nb + i0) * kTile;
@@ -157,6 +158,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const DecArgs a)
     if (tid == 0) {
         *amax_w = 0u;
         *qsum_w = 0;
+        *bad_w = 0;
     }
     // Index state of the product loop, set up here, off the critical path.
     const int r = i0 / a.nb;
@@ -166,20 +168,27 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const DecArgs a)
     const uint4 *qp = qrow + j * 8;
     const uint4 *wl = reinterpret_cast<const uint4 *>(wsm) + lane;
     // Wait for the copies issued above while the previous kernel still runs
-    // (a wait is cheap here and costly after griddepcontrol.wait).
-    bool ok = true;
-    for (int k = 0; k < npre && ok; k++) {
-        int got = 0;
-        if (lane == 0) got = ptx::mbar_wait_sleep(bars + 8u * k, 0u, limit, nullptr, 64) ? 1 : 0;
-        ok = __shfl_sync(0xffffffffu, got, 0) != 0;
+    // (a wait is cheap here and costly after griddepcontrol.wait).  Lanes 0..15
+    // of warp 0 poll warp lane's copies, lane 16 the row scales, sleeping
+    // between tries; the other warps block in the barrier and take no issue
+    // slots from the kernel that shares the SM.
+    __syncwarp();  // lane 0's zeroing of bad_w precedes the other lanes' writes
+    if (warp == 0 && lane <= kWarps) {
+        bool good = true;
+        if (lane < kWarps) {
+            const int wn = (int)(((int64_t)(lane + 1) * n) / kWarps) - (int)(((int64_t)lane * n) / kWarps);
+            const int wc = (wn + kChunk - 1) / kChunk;
+            const int wpre = wc < nslots ? wc : nslots;
+            const uint32_t wb = ptx::smem_u32(smem + a.off_bar) + 8u * (lane * kMaxSlots);
+            for (int k = 0; k < wpre && good; k++) good = ptx::mbar_wait_sleep(wb + 8u * k, 0u, limit, nullptr, 128);
+        } else {
+            good = ptx::mbar_wait_sleep(rbar, 0u, limit, nullptr, 128);
+        }
+        if (!good) *bad_w = 1;
     }
-    if (warp == 0) {
-        int got = 0;
-        if (lane == 0) got = ptx::mbar_wait_sleep(rbar, 0u, limit, nullptr, 64) ? 1 : 0;
-        if (!__shfl_sync(0xffffffffu, got, 0)) ok = false;
-    }
+    __syncthreads();  // copies landed (or bad_w set); acc and the reduction words are zero
+    bool ok = *bad_w == 0;
 
-    __syncthreads();  // acc and the two reduction words are zero for every warp
     asm volatile("griddepcontrol.wait;" ::: "memory");  // x (or q, s) ready; y free
 
     // ---- activations: s, q (permuted) in shared memory, sum(q).
