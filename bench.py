@@ -347,6 +347,7 @@ def run_ours(args, rank, world, dev):
 
     # ---- prefill GEMM (T=2048) ----
     prefill = run_prefill(b, torch, dev, stream, seed)
+    small_batch = run_small_batch(b, torch, dev, stream, seed, weights)
 
     status = b.bitnet_get_device_error(stream.cuda_stream)
     if status != b.BITNET_OK:
@@ -390,6 +391,7 @@ def run_ours(args, rank, world, dev):
                           "how": "bitnet_quant_act + bitnet_w2a8_gemv per linear, same graph replay timing"},
         "gemv_only_ms_per_step": round(gemv_ms_max, 4),
         "prefill": prefill,
+        "small_batch_gemv": small_batch,
         "roofline": roofline,
         "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "ms_per_step": round(e2e_ms, 4),
                 "h2d_bytes_per_step": int(x_host.numel() * 4), "d2h_bytes_per_step": int(y_host.numel() * 4),
@@ -398,6 +400,58 @@ def run_ours(args, rank, world, dev):
         "clocks": clocks.summary(),
     }
     return out
+
+
+SMALL_BATCH = [("o", 2560, 2560), ("gate_up", 13824, 2560), ("wide", 20480, 3200)]
+SMALL_BATCH_B = (1, 4, 16)
+
+
+def run_small_batch(b, torch, dev, stream, seed, weights):
+    """bitnet_w2a8_gemv at B = 1, 4, 16 on the standalone shapes: one call per
+    distinct weight copy (30 copies of the step's O and gate+up weights, 12
+    copies of 20480 x 3200), L2 flushed with a 512 MB write before each timed
+    pass; median of 5 passes, us per call and algorithmic GB/s."""
+    res = {}
+    try:
+        wide = build_weights(b, torch, dev, 12, [("wide", 20480, 3200)], seed ^ 0x99)
+        flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+        for name, o, k in SMALL_BATCH:
+            ws = [wide[(l, name)] for l in range(12)] if name == "wide" else \
+                [weights[(l, name)] for l in range(LAYERS)]
+            res[name] = {"out": o, "K": k}
+            for B in SMALL_BATCH_B:
+                x = torch.randn(B * k, dtype=torch.float32, device=dev)
+                q = torch.empty(B * k, dtype=torch.int8, device=dev)
+                s = torch.empty(B, dtype=torch.float32, device=dev)
+                y = torch.empty(B * o, dtype=torch.float32, device=dev)
+                with torch.cuda.stream(stream):
+                    b.bitnet_quant_act(x, B, k, q, s)
+                    for w in ws:
+                        b.bitnet_w2a8_gemv(w, q, s, B, y)
+                torch.cuda.synchronize(dev)
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=stream):
+                    for w in ws:
+                        b.bitnet_w2a8_gemv(w, q, s, B, y)
+                ms = []
+                for _ in range(5):
+                    with torch.cuda.stream(stream):
+                        flush.fill_(1.0)
+                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    with torch.cuda.stream(stream):
+                        e0.record(stream)
+                        g.replay()
+                        e1.record(stream)
+                    e1.synchronize()
+                    ms.append(e0.elapsed_time(e1) / len(ws))
+                med = sorted(ms)[len(ms) // 2]
+                res[name][f"B{B}"] = {"us": round(med * 1e3, 3),
+                                      "GB/s": round(gemv_bytes(o, k, B) / (med * 1e-3) / 1e9, 1)}
+                del g
+        del flush, wide
+    except Exception as e:  # reported beside the headline, never instead of it
+        res["error"] = f"{type(e).__name__}: {e}"
+    return res
 
 
 def run_prefill(b, torch, dev, stream, seed):

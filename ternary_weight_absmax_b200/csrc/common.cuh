@@ -79,12 +79,13 @@ cudaError_t launch_gemv(const void *data, int64_t rows, int64_t cols, bool unifo
                         const int8_t *q, const float *s, int64_t B, float *y, int32_t *acc,
                         const float *x, int8_t *q_out, float *s_out, const DeviceGlobals &g,
                         cudaStream_t st);
-// Batch-1 decode kernel for uniform rows (decode.cu); launch_gemv picks it when
-// decode_b1_supported says it takes the shape.
-bool decode_b1_supported(int64_t rows, int64_t cols, bool fused);
-cudaError_t launch_decode_b1(const void *data, int64_t rows, int64_t cols, const int8_t *q, const float *s,
-                             float *y, const float *x, int8_t *q_out, float *s_out, const DeviceGlobals &g,
-                             cudaStream_t st);
+// Decode kernels for uniform rows (decode.cu): batch 1 (fused or not) and
+// batches of 2..16 (q and s given); launch_gemv picks them when
+// decode_supported says they take the call.
+bool decode_supported(int64_t rows, int64_t cols, int64_t B, bool fused);
+cudaError_t launch_decode(const void *data, int64_t rows, int64_t cols, int64_t B, const int8_t *q, const float *s,
+                          float *y, const float *x, int8_t *q_out, float *s_out, const DeviceGlobals &g,
+                          cudaStream_t st);
 int absmean_num_partials(int64_t n);
 cudaError_t launch_ternarize(const float *w, int64_t rows, int64_t cols, bool per_block, uint32_t *codes,
                              float *scales, double *partials, float *gamma_slot, cudaStream_t st);

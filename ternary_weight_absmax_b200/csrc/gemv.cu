@@ -1,7 +1,7 @@
 // gemv.cu -- small-batch W2A8 GEMV (1 <= B <= 16) with dp4a: the general
-// kernel (B >= 2, per-block scales, accumulator export, K > 16384).  Batch-1
-// calls on uniform rows go to the decode kernel (decode.cu); launch_gemv at
-// the end of this file chooses.
+// kernel (per-block scales, accumulator export, fused linear at B >= 2,
+// K > 16384).  Calls on uniform rows otherwise go to the decode kernels
+// (decode.cu); launch_gemv at the end of this file chooses.
 //
 // y[b][o] = (sum_j scale[o][j] * acc[b][o][j]) / s[b],
 // acc[b][o][j] = sum_{k in block j} t[o][k] * q[b][k]   (int32, exact).
@@ -472,8 +472,8 @@ cudaError_t launch_gemv(const void *data, int64_t rows, int64_t cols, bool unifo
                         cudaStream_t st) {
     const Layout L = layout_of(rows, cols);
     const char *base = static_cast<const char *>(data);
-    if (B == 1 && uniform && !acc && decode_b1_supported(rows, cols, x != nullptr))
-        return launch_decode_b1(data, rows, cols, q, s, y, x, q_out, s_out, g, st);
+    if (uniform && !acc && decode_supported(rows, cols, B, x != nullptr))
+        return launch_decode(data, rows, cols, B, q, s, y, x, q_out, s_out, g, st);
     Args a;
     a.tiles = reinterpret_cast<const uint4 *>(base + L.off_tiles);
     a.tscales = reinterpret_cast<const float *>(base + L.off_tscales);
