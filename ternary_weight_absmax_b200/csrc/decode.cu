@@ -70,11 +70,11 @@ struct DecArgs {
     int64_t rows;
     int K;
     int nb;
-    int B;         // tokens (batched kernel)
     int tiles_lo;  // every CTA owns tiles_lo or tiles_lo + 1 row tiles
     int extra;     // the first `extra` CTAs own tiles_lo + 1
     int wcap;      // tiles of shared memory per warp: kChunk * (copies in flight), a power of two
     uint32_t off_q, off_acc, off_rsc, off_red, off_bar;
+    int B;         // tokens (batched kernel)
 };
 
 // Shared-memory word of activation word m (bytes 4m .. 4m+3 of q): lane-part t
@@ -247,34 +247,89 @@ struct WeightRing {
     }
 };
 
+// The batch-1 kernel inlines the weight ring's steps (the compiler keeps fewer
+// values live across the products that way: measured 2% faster per step).
 template <bool FUSED, int NX>
 __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const DecArgs a) {
     extern __shared__ __align__(128) unsigned char smem[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int g = lane >> 2, t = lane & 3;
     const int c = blockIdx.x;
+    const int64_t r0 = (int64_t)c * a.tiles_lo + min(c, a.extra);
+    const int nr = a.tiles_lo + (c < a.extra ? 1 : 0);
+    const int n = nr * a.nb;
+    const int i0 = (int)(((int64_t)warp * n) / kWarps);
+    const int nit = (int)(((int64_t)(warp + 1) * n) / kWarps) - i0;
+    const int wcap = a.wcap;  // a power of two, kChunk .. kChunk * kMaxSlots
+    const int nslots = wcap / kChunk;
+    const int nchunks = (nit + kChunk - 1) / kChunk;
+    unsigned char *wsm = smem + (size_t)warp * wcap * kTile;
     uint32_t *qw = reinterpret_cast<uint32_t *>(smem + a.off_q);
     int *acc = reinterpret_cast<int *>(smem + a.off_acc);
     float *rsc = reinterpret_cast<float *>(smem + a.off_rsc);
     unsigned *amax_w = reinterpret_cast<unsigned *>(smem + a.off_red);  // absmax bits (atomic max)
     int *qsum_w = reinterpret_cast<int *>(smem + a.off_red + 4);          // sum(q) (atomic add)
     int *bad_w = reinterpret_cast<int *>(smem + a.off_red + 8);           // a copy wait ran out
+    const uint32_t bars = ptx::smem_u32(smem + a.off_bar) + 8u * (warp * kMaxSlots);
+    const uint32_t rbar = ptx::smem_u32(smem + a.off_bar) + 8u * (kWarps * kMaxSlots);
+    const unsigned char *src = a.tiles + (size_t)(r0 * a.nb + i0) * kTile;
     const uint32_t limit = *a.wait_limit;
-    WeightRing ring;
-    ring.init(a, smem, warp);
 
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
     // ---- before the wait: nothing here depends on the previous kernel.
-    if (lane == 0) ring.start(a, rsc, warp);
-    for (int i = tid; i < ring.nr * kTileRows; i += kThreads) acc[i] = 0;
+    const uint64_t pol = ptx::policy_evict_first();
+    auto issue = [&](int k) {  // lane 0: chunk k of this warp's tiles into its slot
+        const int s = k & (nslots - 1);
+        const uint32_t bytes = (uint32_t)min(kChunk, nit - k * kChunk) * kTile;
+        ptx::mbar_arrive_expect_tx(bars + 8u * s, bytes);
+        ptx::bulk_g2s(ptx::smem_u32(wsm + s * kChunk * kTile), src + (size_t)k * kChunk * kTile, bytes,
+                      bars + 8u * s, pol);
+    };
+    const int npre = nchunks < nslots ? nchunks : nslots;
+    if (lane == 0) {
+        for (int s = 0; s < nslots; s++) ptx::mbar_init(bars + 8u * s, 1);
+        if (warp == 0) ptx::mbar_init(rbar, 1);
+        ptx::fence_mbar_init();
+        for (int k = 0; k < npre; k++) issue(k);
+        if (warp == 0) {
+            const uint32_t bytes = (uint32_t)nr * kTileRows * sizeof(float);
+            ptx::mbar_arrive_expect_tx(rbar, bytes);
+            ptx::bulk_g2s(ptx::smem_u32(rsc), a.rowscale + r0 * kTileRows, bytes, rbar, pol);
+        }
+    }
+    for (int i = tid; i < nr * kTileRows; i += kThreads) acc[i] = 0;
     if (tid == 0) {
         *amax_w = 0u;
         *qsum_w = 0;
         *bad_w = 0;
     }
+    // Index state of the product loop, set up here, off the critical path.
+    const int r = i0 / a.nb;
+    int j = i0 - r * a.nb;
+    int *accp = acc + r * kTileRows + g;  // rows g and g + 8 of the current tile
+    const uint4 *qrow = reinterpret_cast<const uint4 *>(qw + t * 8);  // block 0, this lane's part
+    const uint4 *qp = qrow + j * 8;
+    const uint4 *wl = reinterpret_cast<const uint4 *>(wsm) + lane;
+    // Wait for the copies issued above while the previous kernel still runs
+    // (a wait is cheap here and costly after griddepcontrol.wait).  Lanes 0..15
+    // of warp 0 poll warp lane's copies, lane 16 the row scales, sleeping
+    // between tries; the other warps block in the barrier and take no issue
+    // slots from the kernel that shares the SM.
     __syncwarp();  // lane 0's zeroing of bad_w precedes the other lanes' writes
-    ring.wait_started(a, smem, bad_w, limit, warp, lane);
+    if (warp == 0 && lane <= kWarps) {
+        bool good = true;
+        if (lane < kWarps) {
+            const int wn = (int)(((int64_t)(lane + 1) * n) / kWarps) - (int)(((int64_t)lane * n) / kWarps);
+            const int wc = (wn + kChunk - 1) / kChunk;
+            const int wpre = wc < nslots ? wc : nslots;
+            const uint32_t wb = ptx::smem_u32(smem + a.off_bar) + 8u * (lane * kMaxSlots);
+            for (int k = 0; k < wpre && good; k++) good = ptx::mbar_wait_sleep(wb + 8u * k, 0u, limit, nullptr, 128);
+        } else {
+            good = ptx::mbar_wait_sleep(rbar, 0u, limit, nullptr, 128);
+        }
+        if (!good) *bad_w = 1;
+    }
     __syncthreads();  // copies landed (or bad_w set); acc and the reduction words are zero
     bool ok = *bad_w == 0;
 
@@ -327,12 +382,23 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const DecArgs a)
     if (lane == 0) atomicAdd(qsum_w, qsum);
     __syncthreads();
 
-    // ---- products: the four masked group sums of rows g and g + 8 are held
-    // until the row tile changes.
+    // ---- products.  Items of this warp: i0 .. i0 + nit - 1 (tile r = i / nb,
+    // block j = i % nb), item `it` in shared-memory slot it % wcap; the four
+    // group sums of rows g and g + 8 are held until the tile changes.
     int aA[4] = {0, 0, 0, 0}, aB[4] = {0, 0, 0, 0};
-    const uint4 *qrow = reinterpret_cast<const uint4 *>(qw + t * 8);  // block 0, this lane's part
-    auto item = [&](const uint4 w, int j) {
-        const uint4 *qv = qrow + j * 8;  // qa0 qb0 qa1 qb1 | qa2 qb2 qa3 qb3
+    auto flush = [&]() {
+        const int pA = tig_reduce(combine4(aA));
+        const int pB = tig_reduce(combine4(aB));
+        if (t == 0) {
+            atomicAdd(accp, pA);
+            atomicAdd(accp + 8, pB);
+        }
+#pragma unroll
+        for (int k = 0; k < 4; k++) aA[k] = aB[k] = 0;
+    };
+    // The products of one item: tile word w (lane's 16 bytes), activation
+    // words at qv (qa0 qb0 qa1 qb1 | qa2 qb2 qa3 qb3).
+    auto item = [&](const uint4 w, const uint4 *qv) {
         const uint4 q0 = qv[0], q1 = qv[1];
         const int qa[4] = {(int)q0.x, (int)q0.z, (int)q1.x, (int)q1.z};
         const int qb[4] = {(int)q0.y, (int)q0.w, (int)q1.y, (int)q1.w};
@@ -345,25 +411,78 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const DecArgs a)
             aB[gg] = dp4a_us(w.w & mk, qb[gg], aB[gg]);
         }
     };
-    auto flush = [&](int r) {
-        const int pA = tig_reduce(combine4(aA));
-        const int pB = tig_reduce(combine4(aB));
-        if (t == 0) {
-            atomicAdd(acc + r * kTileRows + g, pA);
-            atomicAdd(acc + r * kTileRows + g + 8, pB);
+    int it = 0;
+    if (nit <= wcap) {
+        // Every tile of the warp is already in shared memory: runs of items
+        // within one row tile, one flush per run.
+        while (it < nit && ok) {
+            const int run = min(nit - it, a.nb - j);
+            const uint4 *wv = wl + it * 32;
+#pragma unroll 2
+            for (int e = 0; e < run; e++) item(wv[e * 32], qp + e * 8);
+            it += run;
+            j += run;
+            qp += run * 8;
+            if (j == a.nb) {
+                flush();
+                accp += kTileRows;
+                j = 0;
+                qp = qrow;
+            }
         }
-#pragma unroll
-        for (int k = 0; k < 4; k++) aA[k] = aB[k] = 0;
-    };
-    ring.run(a, ok, limit, warp, lane, item, flush);
+    } else {
+        // Streaming: item `it` sits in slot it % wcap; chunks from nslots on
+        // are waited for here and refilled as their slots free up.
+        for (; it < nit && ok; it++) {
+            if (it >= wcap && (it & (kChunk - 1)) == 0) {
+                const int k = it / kChunk;
+                int got = 0;
+                if (lane == 0)
+                    got = ptx::mbar_wait(bars + 8u * (k & (nslots - 1)), (uint32_t)(k / nslots) & 1u, limit,
+                                         nullptr) ? 1 : 0;
+                if (!__shfl_sync(0xffffffffu, got, 0)) {
+                    ok = false;
+                    break;
+                }
+            }
+            item(wl[(it & (wcap - 1)) * 32], qp);
+            qp += 8;
+            if (++j == a.nb) {
+                flush();
+                accp += kTileRows;
+                j = 0;
+                qp = qrow;
+            }
+            if ((it & (kChunk - 1)) == kChunk - 1 && it / kChunk + nslots < nchunks) {
+                __syncwarp();  // every lane has read the chunk's slot
+                if (lane == 0) {
+                    ptx::fence_proxy_async_smem();
+                    issue(it / kChunk + nslots);
+                }
+            }
+        }
+    }
+    if (!ok) {
+        // Timed out: record it, then wait out this warp's copies still in flight
+        // (chunks it / kChunk .. the last one issued).
+        if (lane == 0) {
+            atomicOr(a.err, kErrTimeout);
+            const int k0 = it / kChunk;
+            for (int k = k0; k < nchunks && k < k0 + nslots; k++)
+                ptx::mbar_wait(bars + 8u * (k & (nslots - 1)), (uint32_t)(k / nslots) & 1u, kDrainLimit, nullptr);
+            if (warp == 0) ptx::mbar_wait(rbar, 0u, kDrainLimit, nullptr);
+        }
+        __syncwarp();
+    }
+    if (j != 0) flush();  // items since the last tile change (none if j == 0)
     __syncthreads();
 
     const int tot = *qsum_w;  // sum(q) over the row
     // ---- epilogue: y = rowscale * (sum c*q - sum q) * (1/s) in fp32: three
     // roundings, relative error below 2e-7 (the int sum is exact in fp32,
     // |sum| <= 127 * K < 2^22).  The general kernel keeps the fp64 epilogue.
-    for (int i = tid; i < ring.nr * kTileRows; i += kThreads) {
-        const int64_t o = ring.r0 * kTileRows + i;
+    for (int i = tid; i < nr * kTileRows; i += kThreads) {
+        const int64_t o = r0 * kTileRows + i;
         if (o < a.rows) a.y[o] = __fmul_rn(__fmul_rn(rsc[i], int_to_float(acc[i] - tot)), inv_s);
     }
 }
