@@ -348,6 +348,7 @@ def run_ours(args, rank, world, dev):
     # ---- prefill GEMM (T=2048) ----
     prefill = run_prefill(b, torch, dev, stream, seed)
     small_batch = run_small_batch(b, torch, dev, stream, seed, weights)
+    lut = run_lut(b, torch, dev, stream, weights)
 
     status = b.bitnet_get_device_error(stream.cuda_stream)
     if status != b.BITNET_OK:
@@ -392,6 +393,7 @@ def run_ours(args, rank, world, dev):
         "gemv_only_ms_per_step": round(gemv_ms_max, 4),
         "prefill": prefill,
         "small_batch_gemv": small_batch,
+        "lut_gemv_b1": lut,
         "roofline": roofline,
         "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "ms_per_step": round(e2e_ms, 4),
                 "h2d_bytes_per_step": int(x_host.numel() * 4), "d2h_bytes_per_step": int(y_host.numel() * 4),
@@ -449,6 +451,51 @@ def run_small_batch(b, torch, dev, stream, seed, weights):
                                       "GB/s": round(gemv_bytes(o, k, B) / (med * 1e-3) / 1e9, 1)}
                 del g
         del flush, wide
+    except Exception as e:  # reported beside the headline, never instead of it
+        res["error"] = f"{type(e).__name__}: {e}"
+    return res
+
+
+def run_lut(b, torch, dev, stream, weights):
+    """The table-lookup GEMV variant against the dp4a GEMV at batch 1 on the
+    step's four shapes: 30 calls on the 30 layers' weights, one q, L2 flushed
+    before each timed pass, median of 5 passes, us per call."""
+    res = {}
+    try:
+        flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+        for name, o, k in SHAPES:
+            ws = [weights[(l, name)] for l in range(LAYERS)]
+            x = torch.randn(k, dtype=torch.float32, device=dev)
+            q = torch.empty(k, dtype=torch.int8, device=dev)
+            s = torch.empty(1, dtype=torch.float32, device=dev)
+            y = torch.empty(o, dtype=torch.float32, device=dev)
+            calls = {"lut": lambda w: b.bitnet_w2a8_gemv_lut(w, q, s, y),
+                     "dp4a": lambda w: b.bitnet_w2a8_gemv(w, q, s, 1, y)}
+            res[name] = {"out": o, "K": k}
+            for kind, call in calls.items():
+                with torch.cuda.stream(stream):
+                    b.bitnet_quant_act(x, 1, k, q, s)
+                    for w in ws:
+                        call(w)
+                torch.cuda.synchronize(dev)
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=stream):
+                    for w in ws:
+                        call(w)
+                ms = []
+                for _ in range(5):
+                    with torch.cuda.stream(stream):
+                        flush.fill_(1.0)
+                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    with torch.cuda.stream(stream):
+                        e0.record(stream)
+                        g.replay()
+                        e1.record(stream)
+                    e1.synchronize()
+                    ms.append(e0.elapsed_time(e1) / len(ws))
+                res[name][f"{kind}_us"] = round(sorted(ms)[2] * 1e3, 3)
+                del g
+        del flush
     except Exception as e:  # reported beside the headline, never instead of it
         res["error"] = f"{type(e).__name__}: {e}"
     return res

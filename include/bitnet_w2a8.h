@@ -251,6 +251,19 @@ bitnet_status bitnet_w2a8_linear(const bitnet_weight *w, const float *x_dev, int
 bitnet_status bitnet_w2a8_gemm(const bitnet_weight *w, const int8_t *q_dev, const float *s_dev,
                                int64_t T, float *y_dev, bitnet_stream_t stream);
 
+/* Table-lookup variant of bitnet_w2a8_gemv at B = 1, kept for comparison with
+ * the dp4a kernels: the CPU kernels of "浏览器里跑 1-bit 大模型 BitNet
+ * WebAssembly 的 50 倍提速实操" (section "查表（LUT）内核") replace products by
+ * lookups of precomputed activation sub-sums indexed by weight codes; here
+ * each CTA builds, per 128-weight block and byte position, two 16-entry int16
+ * tables over the two weights of a nibble and sums two lookups per byte.
+ * Same arguments and y as bitnet_w2a8_gemv with B = 1 (fp32 epilogue of the
+ * decode kernel).  Errors: NULL, ALIGN, VALUE, UNSUPPORTED (weights without
+ * uniform rows, or K > 8192), CUDA; copy-wait timeouts latch
+ * BITNET_ERR_TIMEOUT. */
+bitnet_status bitnet_w2a8_gemv_lut(const bitnet_weight *w, const int8_t *q_dev, const float *s_dev,
+                                   float *y_dev, bitnet_stream_t stream);
+
 /* Test variants of the two calls above that also write the int32 block
  * accumulators acc_dev[b][o][j], b < B (or T), o < rows, j < cols/128
  * (4-byte aligned), so they can be compared bit for bit. */

@@ -79,6 +79,7 @@ def _load() -> ctypes.CDLL:
         "bitnet_w2a8_linear": ([W, vp, i64, vp, vp, vp, vp], st),
         "bitnet_w2a8_linear_acc": ([W, vp, i64, vp, vp, vp, vp, vp], st),
         "bitnet_w2a8_gemv_acc": ([W, vp, vp, i64, vp, vp, vp], st),
+        "bitnet_w2a8_gemv_lut": ([W, vp, vp, vp, vp], st),
         "bitnet_w2a8_gemm_acc": ([W, vp, vp, i64, vp, vp, vp], st),
         "bitnet_get_device_error": ([vp], st),
         "bitnet_set_wait_limit": ([ctypes.c_uint32], st),
@@ -280,6 +281,12 @@ def bitnet_w2a8_gemv_acc(w: Weight, q, s, B: int, y, acc, stream=None):
                                      B, _dptr(y, "float32", B * w.rows, "y"),
                                      _dptr(acc, "int32", B * w.rows * (w.cols // QK), "acc"), _stream(stream)),
            "bitnet_w2a8_gemv_acc")
+
+
+def bitnet_w2a8_gemv_lut(w: Weight, q, s, y, stream=None):
+    _check(_lib.bitnet_w2a8_gemv_lut(w.ref(), _dptr(q, "int8", w.cols, "q"), _dptr(s, "float32", 1, "s"),
+                                     _dptr(y, "float32", w.rows, "y"), _stream(stream)),
+           "bitnet_w2a8_gemv_lut")
 
 
 def bitnet_w2a8_gemm_acc(w: Weight, q, s, T: int, y, acc, stream=None):

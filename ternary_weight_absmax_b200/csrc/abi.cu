@@ -338,6 +338,24 @@ bitnet_status bitnet_w2a8_gemv_acc(const bitnet_weight *w, const int8_t *q_dev, 
     return gemv_impl(w, q_dev, s_dev, B, y_dev, acc_dev, stream);
 }
 
+bitnet_status bitnet_w2a8_gemv_lut(const bitnet_weight *w, const int8_t *q_dev, const float *s_dev, float *y_dev,
+                                   bitnet_stream_t stream) {
+    t_detail[0] = 0;
+    bitnet_status s = check_weight(w);
+    if (s != BITNET_OK) return s;
+    if (!q_dev || !s_dev || !y_dev) return fail(BITNET_ERR_NULL, "NULL pointer");
+    if (!aligned(q_dev, 16) || !aligned(s_dev, 4) || !aligned(y_dev, 4))
+        return fail(BITNET_ERR_ALIGN, "q needs 16-byte, s/y 4-byte alignment");
+    if (!(w->flags & BITNET_WEIGHT_UNIFORM_ROWS) || w->cols > 8192)
+        return fail(BITNET_ERR_UNSUPPORTED, "the table-lookup GEMV takes uniform rows and K <= 8192");
+    DeviceGlobals g;
+    cudaError_t e = device_globals(&g);
+    if (e != cudaSuccess) return cuda_fail(e, "device globals");
+    e = launch_decode_lut(w->data, w->rows, w->cols, q_dev, s_dev, y_dev, g, reinterpret_cast<cudaStream_t>(stream));
+    if (e == cudaErrorNotSupported) return fail(BITNET_ERR_UNSUPPORTED, "shape not taken by the table-lookup GEMV");
+    return e == cudaSuccess ? BITNET_OK : cuda_fail(e, "gemv_lut launch");
+}
+
 static bitnet_status gemm_impl(const bitnet_weight *w, const int8_t *q_dev, const float *s_dev,
                                int64_t T, float *y_dev, int32_t *acc_dev, bitnet_stream_t stream) {
     t_detail[0] = 0;

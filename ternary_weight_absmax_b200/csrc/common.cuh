@@ -86,6 +86,10 @@ bool decode_supported(int64_t rows, int64_t cols, int64_t B, bool fused);
 cudaError_t launch_decode(const void *data, int64_t rows, int64_t cols, int64_t B, const int8_t *q, const float *s,
                           float *y, const float *x, int8_t *q_out, float *s_out, const DeviceGlobals &g,
                           cudaStream_t st);
+// Table-lookup batch-1 variant (decode.cu), uniform rows, K <= 8192;
+// cudaErrorNotSupported for other shapes.
+cudaError_t launch_decode_lut(const void *data, int64_t rows, int64_t cols, const int8_t *q, const float *s, float *y,
+                              const DeviceGlobals &g, cudaStream_t st);
 int absmean_num_partials(int64_t n);
 cudaError_t launch_ternarize(const float *w, int64_t rows, int64_t cols, bool per_block, uint32_t *codes,
                              float *scales, double *partials, float *gamma_slot, cudaStream_t st);

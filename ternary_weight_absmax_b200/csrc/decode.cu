@@ -602,6 +602,86 @@ __global__ void __launch_bounds__(kThreads, BT >= 8 ? 1 : 2) decode_bn_kernel(co
     }
 }
 
+// Table-lookup variant (batch 1, uniform rows), built for comparison with the
+// dp4a products: the pages' CPU kernels replace multiplications by lookups of
+// precomputed activation sub-sums indexed by weight codes ("浏览器里跑 1-bit
+// 大模型 BitNet WebAssembly 的 50 倍提速实操", section "查表（LUT）内核").
+// Here a nibble of an i2_s byte holds the codes of two weights (columns b and
+// b + 32, or b + 64 and b + 96, of a 128-weight block), so each CTA builds,
+// for every block j and byte position b, two 16-entry tables
+//   T[j][b][h][4 * c1 + c2] = (c1 - 1) * q[128 j + b + 64 h] + (c2 - 1) * q[128 j + b + 32 + 64 h]
+// (code 3 does not occur in repacked weights; its entries are 0) and a lane
+// sums two lookups per weight byte.  The ring, the row-tile ownership and the
+// epilogue are the decode kernel's.
+__global__ void __launch_bounds__(kThreads, 1) decode_lut_kernel(const DecArgs a) {
+    extern __shared__ __align__(128) unsigned char smem[];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int g = lane >> 2, t = lane & 3;
+    int8_t *qn = reinterpret_cast<int8_t *>(smem + a.off_q);                   // [K] natural order
+    int16_t *lut = reinterpret_cast<int16_t *>(smem + a.off_q + a.K);          // [nb][32][2][16]
+    int *acc = reinterpret_cast<int *>(smem + a.off_acc);
+    float *rsc = reinterpret_cast<float *>(smem + a.off_rsc);
+    int *bad_w = reinterpret_cast<int *>(smem + a.off_red);
+    const uint32_t limit = *a.wait_limit;
+    WeightRing ring;
+    ring.init(a, smem, warp);
+
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
+    if (lane == 0) ring.start(a, rsc, warp);
+    for (int i = tid; i < ring.nr * kTileRows; i += kThreads) acc[i] = 0;
+    if (tid == 0) *bad_w = 0;
+    __syncwarp();
+    ring.wait_started(a, smem, bad_w, limit, warp, lane);
+    __syncthreads();
+    bool ok = *bad_w == 0;
+
+    asm volatile("griddepcontrol.wait;" ::: "memory");  // q, s ready; y free
+
+    const int K4 = a.K >> 2;
+    const uint32_t *q4 = reinterpret_cast<const uint32_t *>(a.q);
+    for (int i = tid; i < K4; i += kThreads) reinterpret_cast<uint32_t *>(qn)[i] = q4[i];
+    const float inv_s = __frcp_rn(*a.s);
+    __syncthreads();
+    for (int e = tid; e < a.nb * 32 * 2 * 16; e += kThreads) {
+        const int idx = e & 15, h = (e >> 4) & 1, b = (e >> 5) & 31, j = e >> 10;
+        const int c1 = idx >> 2, c2 = idx & 3;
+        const int qa = qn[128 * j + b + 64 * h], qb = qn[128 * j + b + 32 + 64 * h];
+        lut[e] = (int16_t)((c1 == 3 || c2 == 3) ? 0 : (c1 - 1) * qa + (c2 - 1) * qb);
+    }
+    __syncthreads();
+
+    int sA = 0, sB = 0;
+    // Bytes 4t..4t+3 (words x, y) and 16+4t.. (words z, w) of the block.
+    auto item = [&](const uint4 w, int j) {
+        const int16_t *tj = lut + j * 1024;
+#pragma unroll
+        for (int k = 0; k < 4; k++) {
+            const int b0 = 4 * t + k, b1 = b0 + 16;
+            const int16_t *t0 = tj + b0 * 32, *t1 = tj + b1 * 32;
+            sA += t0[(w.x >> (8 * k + 4)) & 15] + t0[16 + ((w.x >> (8 * k)) & 15)];
+            sB += t0[(w.y >> (8 * k + 4)) & 15] + t0[16 + ((w.y >> (8 * k)) & 15)];
+            sA += t1[(w.z >> (8 * k + 4)) & 15] + t1[16 + ((w.z >> (8 * k)) & 15)];
+            sB += t1[(w.w >> (8 * k + 4)) & 15] + t1[16 + ((w.w >> (8 * k)) & 15)];
+        }
+    };
+    auto flush = [&](int r) {
+        const int pA = tig_reduce(sA), pB = tig_reduce(sB);
+        if (t == 0) {
+            atomicAdd(acc + r * kTileRows + g, pA);
+            atomicAdd(acc + r * kTileRows + g + 8, pB);
+        }
+        sA = sB = 0;
+    };
+    ring.run(a, ok, limit, warp, lane, item, flush);
+    __syncthreads();
+
+    for (int i = tid; i < ring.nr * kTileRows; i += kThreads) {
+        const int64_t o = ring.r0 * kTileRows + i;
+        if (o < a.rows) a.y[o] = __fmul_rn(__fmul_rn(rsc[i], int_to_float(acc[i])), inv_s);
+    }
+}
+
 struct Plan {
     int grid, nx, wcap;
     size_t smem;
@@ -651,6 +731,41 @@ bool plan(const Layout &L, bool fused, int BT, Plan *p) {
     return true;
 }
 
+// Layout for the table-lookup kernel: q in natural order, then the tables
+// (2 KB per 128-weight block); one CTA per SM.
+bool plan_lut(const Layout &L, Plan *p) {
+    const int sms = num_sms();
+    const int grid = (int)(L.ntr < sms ? L.ntr : sms);
+    const int K = (int)L.cols;
+    if (K > 8192) return false;
+    const int64_t lo = L.ntr / grid, hi = lo + (L.ntr % grid ? 1 : 0);
+    const int64_t per_warp = (hi * L.nb + kWarps - 1) / kWarps;
+    int wcap = kChunk;
+    while (wcap < per_warp && wcap < kChunk * kMaxSlots) wcap *= 2;
+    DecArgs &a = p->a;
+    for (;; wcap /= 2) {  // fewer weight slots if the tables need the room
+        a.off_q = (uint32_t)(kWarps * wcap * kTile);
+        a.off_acc = (uint32_t)align_up(a.off_q + (size_t)K + (size_t)L.nb * 2048, 16);
+        a.off_rsc = a.off_acc + (uint32_t)(hi * kTileRows * sizeof(int));
+        a.off_red = a.off_rsc + (uint32_t)(hi * kTileRows * sizeof(float));
+        a.off_bar = a.off_red + 128;
+        p->smem = a.off_bar + 8 * (kWarps * kMaxSlots + 1);
+        if (p->smem <= 200 * 1024) break;
+        if (wcap == kChunk) return false;
+    }
+    a.rows = L.rows;
+    a.K = K;
+    a.nb = (int)L.nb;
+    a.B = 1;
+    a.tiles_lo = (int)lo;
+    a.extra = (int)(L.ntr % grid);
+    a.wcap = wcap;
+    p->grid = grid;
+    p->nx = 1;
+    p->wcap = wcap;
+    return true;
+}
+
 int batch_tile(int64_t B) { return B <= 1 ? 1 : B <= 2 ? 2 : B <= 4 ? 4 : B <= 8 ? 8 : 16; }
 
 template <class Kernel>
@@ -694,6 +809,27 @@ cudaError_t run_bn(const Plan &p, cudaStream_t st) {
 }
 
 }  // namespace
+
+cudaError_t launch_decode_lut(const void *data, int64_t rows, int64_t cols, const int8_t *q, const float *s, float *y,
+                              const DeviceGlobals &g, cudaStream_t st) {
+    const Layout L = layout_of(rows, cols);
+    Plan p;
+    if (!plan_lut(L, &p)) return cudaErrorNotSupported;
+    const unsigned char *base = static_cast<const unsigned char *>(data);
+    DecArgs &a = p.a;
+    a.tiles = base + L.off_tiles;
+    a.rowscale = reinterpret_cast<const float *>(base + L.off_rowscale);
+    a.q = q;
+    a.s = s;
+    a.x = nullptr;
+    a.q_out = nullptr;
+    a.s_out = nullptr;
+    a.y = y;
+    a.err = g.err;
+    a.wait_limit = g.wait_limit;
+    static bool configured[64];
+    return launch(decode_lut_kernel, configured, p, st);
+}
 
 bool decode_supported(int64_t rows, int64_t cols, int64_t B, bool fused) {
     Plan p;

@@ -118,6 +118,15 @@ def test_device_calls_validate_before_touching_the_gpu(b):
     w.cols = 128
     assert lib.bitnet_w2a8_gemm(ctypes.byref(w), 16, 16, -1, 16, None) == b.BITNET_ERR_SHAPE
     assert lib.bitnet_w2a8_gemm(ctypes.byref(w), 16, 16, 0, 16, None) == b.BITNET_OK  # T=0: no-op
+    # Table-lookup GEMV: NULL / alignment, then weights without uniform rows or K > 8192.
+    assert lib.bitnet_w2a8_gemv_lut(ctypes.byref(w), None, 16, 16, None) == b.BITNET_ERR_NULL
+    assert lib.bitnet_w2a8_gemv_lut(ctypes.byref(w), 17, 16, 16, None) == b.BITNET_ERR_ALIGN
+    w.flags = 0
+    assert lib.bitnet_w2a8_gemv_lut(ctypes.byref(w), 16, 16, 16, None) == b.BITNET_ERR_UNSUPPORTED
+    w.flags = b.BITNET_WEIGHT_UNIFORM_ROWS
+    w.cols = 8320
+    assert lib.bitnet_w2a8_gemv_lut(ctypes.byref(w), 16, 16, 16, None) == b.BITNET_ERR_UNSUPPORTED
+    w.cols = 128
     assert lib.bitnet_w2a8_gemm(ctypes.byref(w), 16, 16, 4, 8, None) == b.BITNET_ERR_ALIGN
     assert lib.bitnet_quant_act(16, 1, 100, 16, 16, None, None) == b.BITNET_ERR_SHAPE
     assert lib.bitnet_quant_act(16, 0, 128, 16, 16, None, None) == b.BITNET_OK

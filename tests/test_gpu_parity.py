@@ -458,3 +458,55 @@ def test_linear_full_size_sampled_rows(rows, K, B):
         assert_decode_close(y[:, pick], ref, f"decode linear {rows}x{K}")
     else:
         np.testing.assert_array_equal(y[:, pick], ref)
+
+
+# ------------------------------------------------ table-lookup GEMV variant --
+
+def _run_lut(t, sc, x, guard=64):
+    b = lib()
+    tt = torch()
+    rows, K = t.shape
+    w, _ = device_weight(t, sc)
+    q, s, _ = gpu_quant(x)
+    ybuf = tt.full((rows + 2 * guard,), 12345.0, dtype=tt.float32, device="cuda")
+    y = ybuf[guard:guard + rows]
+    b.bitnet_w2a8_gemv_lut(w, q, s, y)
+    assert b.bitnet_get_device_error() == b.BITNET_OK
+    yb = to_np(ybuf)
+    assert np.all(yb[:guard] == 12345.0) and np.all(yb[guard + rows:] == 12345.0), "output guard overwritten"
+    return to_np(q).reshape(1, K), to_np(s), to_np(y).reshape(1, rows)
+
+
+@pytest.mark.parametrize("rows,K,mode", [
+    (256, 512, "tensor"), (1, 128, "tensor"), (17, 256, "row"), (300, 1024, "tensor"), (777, 1280, "row"),
+    (3840, 2560, "tensor"), (2560, 6912, "tensor"), (4096, 8192, "tensor"), (7109, 640, "tensor"),
+])
+def test_lut_gemv_matches_oracle(rows, K, mode):
+    t, sc, x = _gemv_case(rows, K, 1, mode, seed=rows * 7 + K)
+    q, s, y = _run_lut(t, sc, x)
+    rq, rs, _ = oracle.quant_act(x)
+    np.testing.assert_array_equal(q, rq)
+    assert_decode_close(y, oracle.linear(oracle.pack_i2s(t), sc, K, rq, rs), f"lut {rows}x{K}")
+
+
+def test_lut_gemv_full_size_sampled_rows():
+    rows, K = 13824, 2560
+    t, sc, x = _gemv_case(rows, K, 1, "tensor", seed=4711)
+    q, s, y = _run_lut(t, sc, x)
+    rq, rs, _ = oracle.quant_act(x)
+    pick = np.unique(np.concatenate([[0, rows - 1], syn.splitmix64(rows, np.arange(60)) % np.uint64(rows)]))
+    pick = pick.astype(np.int64)
+    ref = oracle.linear(oracle.pack_i2s(t[pick]), sc[pick], K, rq, rs)
+    assert_decode_close(y[:, pick], ref, "lut full size")
+
+
+def test_lut_gemv_rejects_block_scales():
+    b = lib()
+    tt = torch()
+    t, sc, x = _gemv_case(64, 512, 1, "block", seed=5)
+    w, _ = device_weight(t, sc)
+    q, s, _ = gpu_quant(x)
+    y = tt.empty(64, dtype=tt.float32, device="cuda")
+    with pytest.raises(b.BitnetError) as e:
+        b.bitnet_w2a8_gemv_lut(w, q, s, y)
+    assert e.value.status == b.BITNET_ERR_UNSUPPORTED
