@@ -42,6 +42,10 @@
 // Integer sums are exact, so the atomics leave the result independent of
 // their order.  Every wait on a copy is bounded; on a timeout the kernel sets
 // the device error word, waits (bounded) for its copies in flight and returns.
+//
+// Two more kernels share the weight ring (WeightRing below): the batched
+// kernel for 2..16 tokens (decode_bn_kernel) and a table-lookup variant for
+// comparison (decode_lut_kernel).
 #include "common.cuh"
 #include "dp4a.cuh"
 #include "tcgen05.cuh"
