@@ -772,8 +772,10 @@ bool plan_lut(const Layout &L, Plan *p) {
 
 int batch_tile(int64_t B) { return B <= 1 ? 1 : B <= 2 ? 2 : B <= 4 ? 4 : B <= 8 ? 8 : 16; }
 
+// smem_cap: the kernel's dynamic shared-memory opt-in (the most any of its
+// plans asks for: 100 KB for two CTAs per SM, 200 KB for one).
 template <class Kernel>
-cudaError_t launch(Kernel k, bool *configured, const Plan &p, cudaStream_t st) {
+cudaError_t launch(Kernel k, bool *configured, int smem_cap, const Plan &p, cudaStream_t st) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
@@ -783,7 +785,7 @@ cudaError_t launch(Kernel k, bool *configured, const Plan &p, cudaStream_t st) {
         // consecutive linears can share an SM without it being reconfigured.
         e = cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
         if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+            e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_cap);
         if (e != cudaSuccess) return e;
         configured[dev] = true;
     }
@@ -803,13 +805,13 @@ cudaError_t launch(Kernel k, bool *configured, const Plan &p, cudaStream_t st) {
 template <bool FUSED, int NX>
 cudaError_t run_b1(const Plan &p, cudaStream_t st) {
     static bool configured[64];
-    return launch(decode_b1_kernel<FUSED, NX>, configured, p, st);
+    return launch(decode_b1_kernel<FUSED, NX>, configured, 100 * 1024, p, st);
 }
 
 template <int BT>
 cudaError_t run_bn(const Plan &p, cudaStream_t st) {
     static bool configured[64];
-    return launch(decode_bn_kernel<BT>, configured, p, st);
+    return launch(decode_bn_kernel<BT>, configured, BT >= 8 ? 200 * 1024 : 100 * 1024, p, st);
 }
 
 }  // namespace
@@ -832,7 +834,7 @@ cudaError_t launch_decode_lut(const void *data, int64_t rows, int64_t cols, cons
     a.err = g.err;
     a.wait_limit = g.wait_limit;
     static bool configured[64];
-    return launch(decode_lut_kernel, configured, p, st);
+    return launch(decode_lut_kernel, configured, 200 * 1024, p, st);
 }
 
 bool decode_supported(int64_t rows, int64_t cols, int64_t B, bool fused) {
