@@ -214,13 +214,13 @@ bitnet_status bitnet_quant_act(const float *x_dev, int64_t T, int64_t K, int8_t 
  * with acc the int32 block dot products of the ternary weights and q.
  * q_dev: B*K int8 (16-byte aligned); s_dev: B fp32; y_dev: B*rows fp32
  * (4-byte aligned).  The int32 sums are exact.  The sum over blocks runs in
- * fp64 and is rounded once to fp32, except for B = 1 on weights with uniform
- * rows (BITNET_WEIGHT_UNIFORM_ROWS, the per-tensor absmean case) and
- * K <= 16384, the token-by-token decode call: there y = scale * acc * (1/s)
- * in fp32 (three roundings, within 2.4e-7 relative of the fp64 value).
+ * fp64 and is rounded once to fp32, except on weights with uniform rows
+ * (BITNET_WEIGHT_UNIFORM_ROWS, the per-tensor absmean case) and K <= 16384,
+ * the decode calls: there y = scale * acc * (1/s) in fp32 (three roundings,
+ * within 2.4e-7 relative of the fp64 value).
  * Errors: NULL, SHAPE (B outside 1..16, K mismatch), ALIGN, VALUE (w not
- * repacked), CUDA.  The batch-1 decode kernel waits (bounded) on its weight
- * copies; a wait that runs out latches BITNET_ERR_TIMEOUT.
+ * repacked), CUDA.  The decode kernels wait (bounded) on their weight copies;
+ * a wait that runs out latches BITNET_ERR_TIMEOUT.
  * The GEMV, the fused linear and the quantiser use programmatic dependent
  * launch: a GEMV may start reading its (constant) weights while the kernel
  * before it on the stream is still running, and reads q, s (or x) and writes
@@ -235,8 +235,8 @@ bitnet_status bitnet_w2a8_gemv(const bitnet_weight *w, const int8_t *q_dev, cons
  * shared memory).  x_dev: B*K fp32 (16-byte aligned); y_dev: B*rows fp32.
  * q_out_dev (B*K int8) and s_out_dev (B fp32) are optional (NULL = not
  * written; 4-byte aligned) and receive the quantised activations.  The fp32
- * epilogue of the batch-1 decode case is the GEMV's (B = 1, uniform rows,
- * K <= 16384).
+ * epilogue is the GEMV's at B = 1 on uniform rows with K <= 16384; at
+ * B >= 2 this call runs the general kernel (fp64 epilogue).
  * Errors: NULL, SHAPE, ALIGN, VALUE, BUFSIZE, CUDA; BITNET_ERR_TIMEOUT is
  * latched as for the GEMV. */
 bitnet_status bitnet_w2a8_linear(const bitnet_weight *w, const float *x_dev, int64_t B, float *y_dev,
