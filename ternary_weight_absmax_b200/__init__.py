@@ -55,7 +55,7 @@ class bitnet_weight(ctypes.Structure):
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError(f"libbitnet_w2a8.so is not built ({LIB_PATH}); run __graft_entry__.build() "
-                          "or python -m ternary_weight_absmax_b200._build_lib")
+                          "or python ternary_weight_absmax_b200/_build_lib.py")
     lib = ctypes.CDLL(LIB_PATH)
     i64, sz, vp, st = ctypes.c_int64, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_int
     W = ctypes.POINTER(bitnet_weight)
