@@ -90,65 +90,101 @@ def aggregate(per_rank_ms, per_rank_bytes):
 # --------------------------------------------------------------- clocks --
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+    """SM clock, power and clock-event (throttle) reasons sampled every 100 ms
+    through NVML (read-only queries) while the timed region runs.  The device is
+    found by its UUID, so the index under CUDA_VISIBLE_DEVICES does not matter.
+    Falls back to `nvidia-smi -lms` with line-buffered output if NVML cannot be
+    loaded (a fully buffered pipe loses every sample when the tool is stopped)."""
 
-    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = (("hw_slowdown", 0x8), ("sw_thermal_slowdown", 0x20), ("hw_thermal_slowdown", 0x40),
+               ("hw_power_brake_slowdown", 0x80), ("sw_power_cap", 0x4))
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active")
 
-    def __init__(self, index: int):
-        self.index = index
-        self.proc = None
-        self.lines = []
+    def __init__(self, device):
+        self.device = device
+        self.samples = []  # (time, sm_mhz, max_mhz, power_w, reasons bitmask)
         self.t0 = self.t1 = None
+        self._stop = threading.Event()
+        self._thread = None
+        self._proc = None
+        self.source = "none"
+
+    def _nvml_handle(self):
+        import pynvml
+        import torch
+        pynvml.nvmlInit()
+        props = torch.cuda.get_device_properties(self.device)
+        try:
+            return pynvml, pynvml.nvmlDeviceGetHandleByUUID("GPU-" + str(props.uuid))
+        except pynvml.NVMLError:
+            bus = f"{props.pci_domain_id:08X}:{props.pci_bus_id:02X}:{props.pci_device_id:02X}.0"
+            return pynvml, pynvml.nvmlDeviceGetHandleByPciBusId(bus)
 
     def start(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            threading.Thread(target=self._read, daemon=True).start()
-        except OSError:
-            self.proc = None
+            nv, h = self._nvml_handle()
+            mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+            self.source = "nvml"
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append((time.time(), line.strip()))
+            def run():
+                while not self._stop.is_set():
+                    try:
+                        self.samples.append((time.time(), nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM), mx,
+                                             nv.nvmlDeviceGetPowerUsage(h) / 1000.0,
+                                             nv.nvmlDeviceGetCurrentClocksEventReasons(h)))
+                    except nv.NVMLError:
+                        pass
+                    self._stop.wait(0.1)
+            self._thread = threading.Thread(target=run, daemon=True)
+            self._thread.start()
+            return
+        except Exception:
+            pass
+        try:
+            import torch
+            idx = str(torch.cuda.get_device_properties(self.device).uuid)
+            self._proc = subprocess.Popen(
+                ["stdbuf", "-oL", "nvidia-smi", "-i", "GPU-" + idx, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.source = "nvidia-smi"
+
+            def read():
+                for line in self._proc.stdout:
+                    p = [x.strip() for x in line.split(",")]
+                    try:
+                        self.samples.append((time.time(), float(p[0]), float(p[1]), float(p[2]), int(p[3], 16)))
+                    except (ValueError, IndexError):
+                        continue
+            self._thread = threading.Thread(target=read, daemon=True)
+            self._thread.start()
+        except (OSError, RuntimeError):
+            self._proc = None
 
     def mark(self, which):
         setattr(self, which, time.time())
 
     def stop(self):
-        if self.proc:
-            self.proc.terminate()
+        self._stop.set()
+        if self._proc:
+            self._proc.terminate()
             try:
-                self.proc.wait(timeout=5)
+                self._proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
-                self.proc.kill()
+                self._proc.kill()
+        if self._thread:
+            self._thread.join(timeout=2)
 
     def summary(self):
-        rows = [l for ts, l in self.lines if self.t0 is None or (self.t0 - 0.25 <= ts <= self.t1 + 0.25)]
+        rows = [r for r in self.samples if self.t0 is None or (self.t0 <= r[0] <= (self.t1 or r[0]))]
         if not rows:
-            rows = [l for _, l in self.lines]
-        mhz, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for l in rows:
-            p = [x.strip() for x in l.split(",")]
-            if len(p) < 9:
-                continue
-            try:
-                mhz.append(float(p[1]))
-                mx = float(p[2])
-            except ValueError:
-                continue
-            for n, v in zip(names, p[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        if not mhz:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
-        mhz.sort()
-        return {"sm_mhz": mhz[len(mhz) // 2], "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(mhz)}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0,
+                    "source": self.source}
+        mhz = sorted(r[1] for r in rows)
+        reasons = sorted({n for r in rows for n, bit in self.REASONS if r[4] & bit})
+        return {"sm_mhz": mhz[len(mhz) // 2], "sm_min_mhz": mhz[0], "sm_max_mhz": rows[-1][2],
+                "power_w_median": sorted(r[3] for r in rows)[len(rows) // 2], "reasons": reasons,
+                "samples": len(rows), "source": self.source}
 
 
 # ----------------------------------------------------------- our arm --
@@ -290,7 +326,7 @@ def run_ours(args, rank, world, dev):
             ms.append(e0.elapsed_time(e1))
         return ms
 
-    clocks = ClockSampler(torch.cuda.current_device() if isinstance(dev, int) else dev.index or 0)
+    clocks = ClockSampler(dev)
     clocks.start()
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):

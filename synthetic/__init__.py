@@ -107,3 +107,16 @@ def positive_scales(seed: int, rows: int, nb: int, uniform_per_row: bool = False
     if uniform_per_row:
         return np.repeat(v[:, None], nb, axis=1)
     return v.reshape(rows, nb)
+
+
+def integer_rows(seed: int, T: int, K: int, peak: int = 127) -> np.ndarray:
+    """fp32 rows [T][K] of integers drawn uniformly from [-peak, peak], with
+    element (t, splitmix64 pick) of every row set to +-peak, so each row's
+    largest magnitude is exactly `peak`."""
+    z = splitmix64(seed, np.arange(T * K, dtype=np.uint64))
+    x = ((z % np.uint64(2 * peak + 1)).astype(np.int64) - peak).reshape(T, K)
+    pick = splitmix64(seed ^ 0x5EED, np.arange(T, dtype=np.uint64))
+    col = (pick % np.uint64(K)).astype(np.int64)
+    sign = np.where((pick >> np.uint64(32)) & np.uint64(1), -1, 1)
+    x[np.arange(T), col] = sign * peak
+    return x.astype(np.float32)

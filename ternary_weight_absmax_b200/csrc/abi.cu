@@ -5,6 +5,7 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "common.cuh"
@@ -90,15 +91,15 @@ cudaError_t device_globals(DeviceGlobals *out) {
 }
 
 int num_sms() {
-    static int n[64];
+    static std::atomic<int> n[64];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-    if (!n[dev]) {
-        int v = 0;
+    int v = n[dev].load(std::memory_order_relaxed);
+    if (!v) {
         if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) v = 148;
-        n[dev] = v;
+        n[dev].store(v, std::memory_order_relaxed);
     }
-    return n[dev];
+    return v;
 }
 
 }  // namespace bitnet

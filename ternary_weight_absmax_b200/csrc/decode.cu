@@ -3,10 +3,11 @@
 //
 // y[o] = rowscale[o] * (sum_k t[o][k] * q[k]) / s,   q = per-token absmax int8
 // activations ("5倍性能跃升：BitNet与llama.cpp的1-bit LLM推理架构对决", section
-// "GPU内核突破": 2-bit weights x 8-bit activations with dp4a; the activation
-// quantisation is the per-token absmax of "BitNet b1.58", section "Quantization
-// Function").  q and the integer sums are exactly those of the general kernel;
-// the epilogue runs in fp32 (below).
+// "GPU内核突破": 2-bit weights x 8-bit activations with dp4a).  The pages do not
+// print the activation formula; the library reads it as s = 127 / max(absmax,
+// 1e-5) and q = rint(x * s), ties to even (one fp32 multiply), the reading the
+// quantiser documents.  q and the integer sums are exactly those of the general
+// kernel; the epilogue runs in fp32 (below).
 //
 // A decode step is a chain of dependent linears of a few microseconds each, so
 // what costs is the chain's latency: the time from the previous kernel's end
@@ -46,6 +47,8 @@
 // Two more kernels share the weight ring (WeightRing below): the batched
 // kernel for 2..16 tokens (decode_bn_kernel) and a table-lookup variant for
 // comparison (decode_lut_kernel).
+#include <atomic>
+
 #include "common.cuh"
 #include "dp4a.cuh"
 #include "tcgen05.cuh"
@@ -164,7 +167,9 @@ struct WeightRing {
     // Lanes 0..15 of warp 0 wait for warp lane's first copies, lane 16 for the
     // row scales, sleeping between polls while the other warps block in the
     // barrier that follows (they take no issue slots from the kernel sharing
-    // the SM).  A wait that runs out sets *bad.
+    // the SM).  A wait that runs out sets *bad.  Call only after a CTA barrier
+    // that follows every warp's start(): the barriers polled here belong to
+    // other warps.
     __device__ __forceinline__ void wait_started(const DecArgs &a, unsigned char *smem, int *bad, uint32_t limit,
                                                  int warp, int lane) const {
         if (warp != 0 || lane > kWarps) return;
@@ -319,8 +324,11 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const DecArgs a)
     // (a wait is cheap here and costly after griddepcontrol.wait).  Lanes 0..15
     // of warp 0 poll warp lane's copies, lane 16 the row scales, sleeping
     // between tries; the other warps block in the barrier and take no issue
-    // slots from the kernel that shares the SM.
-    __syncwarp();  // lane 0's zeroing of bad_w precedes the other lanes' writes
+    // slots from the kernel that shares the SM.  The barrier first: every
+    // warp's lane 0 has initialised its slot barriers (and issued its copies)
+    // before warp 0 polls them -- shared memory left by an earlier CTA could
+    // otherwise look like a completed phase -- and bad_w is zero.
+    __syncthreads();
     if (warp == 0 && lane <= kWarps) {
         bool good = true;
         if (lane < kWarps) {
@@ -519,7 +527,7 @@ __global__ void __launch_bounds__(kThreads, BT >= 8 ? 1 : 2) decode_bn_kernel(co
     for (int i = tid; i < ring.nr * kTileRows * BT; i += kThreads) acc[i] = 0;
     if (tid < BT) qsum_w[tid] = 0;
     if (tid == 0) *bad_w = 0;
-    __syncwarp();
+    __syncthreads();  // every warp's slot barriers are initialised before warp 0 polls them
     ring.wait_started(a, smem, bad_w, limit, warp, lane);
     __syncthreads();
     bool ok = *bad_w == 0;
@@ -635,7 +643,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_lut_kernel(const DecArgs a
     if (lane == 0) ring.start(a, rsc, warp);
     for (int i = tid; i < ring.nr * kTileRows; i += kThreads) acc[i] = 0;
     if (tid == 0) *bad_w = 0;
-    __syncwarp();
+    __syncthreads();  // every warp's slot barriers are initialised before warp 0 polls them
     ring.wait_started(a, smem, bad_w, limit, warp, lane);
     __syncthreads();
     bool ok = *bad_w == 0;
@@ -775,19 +783,21 @@ int batch_tile(int64_t B) { return B <= 1 ? 1 : B <= 2 ? 2 : B <= 4 ? 4 : B <= 8
 // smem_cap: the kernel's dynamic shared-memory opt-in (the most any of its
 // plans asks for: 100 KB for two CTAs per SM, 200 KB for one).
 template <class Kernel>
-cudaError_t launch(Kernel k, bool *configured, int smem_cap, const Plan &p, cudaStream_t st) {
+cudaError_t launch(Kernel k, std::atomic<bool> *configured, int smem_cap, const Plan &p, cudaStream_t st) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    if (!configured[dev]) {
+    // Two host threads may both configure a kernel the first time; setting the
+    // same attributes twice is harmless, and the flag itself is atomic.
+    if (!configured[dev].load(std::memory_order_acquire)) {
         // Every launch asks for the same shared-memory carveout, so CTAs of
         // consecutive linears can share an SM without it being reconfigured.
         e = cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
         if (e == cudaSuccess)
             e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_cap);
         if (e != cudaSuccess) return e;
-        configured[dev] = true;
+        configured[dev].store(true, std::memory_order_release);
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)p.grid);
@@ -804,13 +814,13 @@ cudaError_t launch(Kernel k, bool *configured, int smem_cap, const Plan &p, cuda
 
 template <bool FUSED, int NX>
 cudaError_t run_b1(const Plan &p, cudaStream_t st) {
-    static bool configured[64];
+    static std::atomic<bool> configured[64];
     return launch(decode_b1_kernel<FUSED, NX>, configured, 100 * 1024, p, st);
 }
 
 template <int BT>
 cudaError_t run_bn(const Plan &p, cudaStream_t st) {
-    static bool configured[64];
+    static std::atomic<bool> configured[64];
     return launch(decode_bn_kernel<BT>, configured, BT >= 8 ? 200 * 1024 : 100 * 1024, p, st);
 }
 
@@ -833,7 +843,7 @@ cudaError_t launch_decode_lut(const void *data, int64_t rows, int64_t cols, cons
     a.y = y;
     a.err = g.err;
     a.wait_limit = g.wait_limit;
-    static bool configured[64];
+    static std::atomic<bool> configured[64];
     return launch(decode_lut_kernel, configured, 200 * 1024, p, st);
 }
 

@@ -14,6 +14,8 @@
 // Bound: HBM for prefill-sized T (4 B read + 1 B written per element), launch
 // latency for decode.  Launched with programmatic dependent launch so the
 // next kernel (the GEMV) can start streaming its weights meanwhile.
+#include <atomic>
+
 #include "common.cuh"
 
 namespace bitnet {
@@ -89,12 +91,12 @@ quant_act_kernel(const float4 *__restrict__ x, int64_t K, int8_t *__restrict__ q
 cudaError_t launch_quant_act(const float *x, int64_t T, int64_t K, int8_t *q, float *s,
                              int32_t *blocksum, cudaStream_t st) {
     if (T == 0) return cudaSuccess;
-    static bool configured[64];
+    static std::atomic<bool> configured[64];  // set once per device; a repeat is harmless
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    if (!configured[dev]) {
+    if (!configured[dev].load(std::memory_order_acquire)) {
         // Same shared-memory carveout as the decode kernel, so the two can share
         // an SM under programmatic dependent launch without a reconfiguration.
         for (auto k : {quant_act_kernel<true>, quant_act_kernel<false>}) {
@@ -102,7 +104,7 @@ cudaError_t launch_quant_act(const float *x, int64_t T, int64_t K, int8_t *q, fl
                                      cudaSharedmemCarveoutMaxShared);
             if (e != cudaSuccess) return e;
         }
-        configured[dev] = true;
+        configured[dev].store(true, std::memory_order_release);
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)T);
