@@ -242,6 +242,56 @@ bitnet_status bitnet_w2a8_gemv(const bitnet_weight *w, const int8_t *q_dev, cons
 bitnet_status bitnet_w2a8_linear(const bitnet_weight *w, const float *x_dev, int64_t B, float *y_dev,
                                  int8_t *q_out_dev, float *s_out_dev, bitnet_stream_t stream);
 
+/* A sequence of batch-1 decode linears in ONE persistent kernel.  Each entry
+ * computes exactly what bitnet_w2a8_linear computes with B = 1 on uniform rows
+ * (same q, s, int32 sums and fp32 epilogue, bit for bit): per-token absmax
+ * int8 quantisation of x ("5倍性能跃升：BitNet与llama.cpp的1-bit LLM推理架构
+ * 对决", section "GPU内核突破": 8-bit activations, 2-bit weights), the
+ * integer add / subtract / skip product ("BitRun v0.2 实测", section
+ * "三值权重与 1.58-bit 的由来") and y = rowscale * sum * (1/s).  Batch-1
+ * decode reads every weight once and is bound by memory bandwidth ("浏览器里跑
+ * 1-bit 大模型 BitNet WebAssembly 的 50 倍提速实操", section "为什么是 WASM");
+ * one kernel for the whole list keeps the weights streaming from HBM with no
+ * gap between linears, where one launch per linear pays a launch, an
+ * activation phase and a tail each.
+ *
+ * wait_for = -1: x is ready when the call is enqueued (it may be written by
+ * earlier work on `stream`).  wait_for = j (0 <= j < this entry's index): x is
+ * (part of) the y of entry j, and this linear's products wait, on the device,
+ * until every output of entry j is written.  Linears that wait for nothing
+ * run concurrently; a chain of waits runs one linear after another.
+ * Memory rules (checked on the host; BITNET_ERR_VALUE otherwise): no two y
+ * ranges overlap, and an x range may overlap a y range only of an entry it
+ * waits for directly or through a chain of waits, or of an entry that waits
+ * (directly or through a chain) for it (in-place reuse of a buffer once read).
+ * w: repacked, BITNET_WEIGHT_UNIFORM_ROWS, cols <= BITNET_SEQ_MAX_COLS; x_dev
+ * [cols] fp32, 16-byte aligned; y_dev [rows] fp32, 4-byte aligned.
+ * workspace_dev: device memory of at least
+ * bitnet_w2a8_linear_seq_workspace_bytes(n) bytes, 4-byte aligned, caller
+ * owned, ZERO-FILLED before its first use; every call leaves it zeroed.  It
+ * may be NULL (and workspace_bytes 0) when no entry waits.  Calls that share
+ * a workspace must not overlap on the GPU.  A call with waits is a
+ * cooperative launch (one CTA per SM, all resident); it fails with
+ * BITNET_ERR_CUDA if the device cannot co-schedule them.
+ * Errors: NULL, SHAPE (n outside 1..BITNET_SEQ_MAX_LINEARS), ALIGN, VALUE
+ * (bad wait_for, not repacked, overlapping buffers), UNSUPPORTED (rows not
+ * uniform, or cols > BITNET_SEQ_MAX_COLS), BUFSIZE (workspace), CUDA.  Bounded
+ * device waits (copies, producers) that run out latch BITNET_ERR_TIMEOUT. */
+#define BITNET_SEQ_MAX_LINEARS 256
+#define BITNET_SEQ_MAX_COLS 16384
+
+typedef struct {
+    const bitnet_weight *w;
+    const float *x_dev;
+    float *y_dev;
+    int32_t wait_for;
+} bitnet_linear_desc;
+
+size_t bitnet_w2a8_linear_seq_workspace_bytes(int32_t n);
+
+bitnet_status bitnet_w2a8_linear_seq(const bitnet_linear_desc *list, int32_t n, void *workspace_dev,
+                                     size_t workspace_bytes, bitnet_stream_t stream);
+
 /* Prefill GEMM, T >= 1 tokens, same result as the GEMV (tcgen05 int8
  * tensor cores, int32 accumulators in tensor memory).
  * q_dev: T*K int8 (16-byte aligned); s_dev: T fp32; y_dev: T*rows fp32

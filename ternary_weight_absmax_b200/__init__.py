@@ -52,6 +52,15 @@ class bitnet_weight(ctypes.Structure):
                 ("flags", ctypes.c_uint32)]
 
 
+class bitnet_linear_desc(ctypes.Structure):
+    _fields_ = [("w", ctypes.POINTER(bitnet_weight)), ("x_dev", ctypes.c_void_p), ("y_dev", ctypes.c_void_p),
+                ("wait_for", ctypes.c_int32)]
+
+
+BITNET_SEQ_MAX_LINEARS = 256
+BITNET_SEQ_MAX_COLS = 16384
+
+
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError(f"libbitnet_w2a8.so is not built ({LIB_PATH}); run __graft_entry__.build() "
@@ -81,6 +90,8 @@ def _load() -> ctypes.CDLL:
         "bitnet_w2a8_gemv_acc": ([W, vp, vp, i64, vp, vp, vp], st),
         "bitnet_w2a8_gemv_lut": ([W, vp, vp, vp, vp], st),
         "bitnet_w2a8_gemm_acc": ([W, vp, vp, i64, vp, vp, vp], st),
+        "bitnet_w2a8_linear_seq_workspace_bytes": ([ctypes.c_int32], sz),
+        "bitnet_w2a8_linear_seq": ([ctypes.POINTER(bitnet_linear_desc), ctypes.c_int32, vp, sz, vp], st),
         "bitnet_get_device_error": ([vp], st),
         "bitnet_set_wait_limit": ([ctypes.c_uint32], st),
     }
@@ -294,6 +305,29 @@ def bitnet_w2a8_gemm_acc(w: Weight, q, s, T: int, y, acc, stream=None):
                                      T, _dptr(y, "float32", T * w.rows, "y"),
                                      _dptr(acc, "int32", T * w.rows * (w.cols // QK), "acc"), _stream(stream)),
            "bitnet_w2a8_gemm_acc")
+
+
+def bitnet_w2a8_linear_seq_workspace_bytes(n: int) -> int:
+    return _lib.bitnet_w2a8_linear_seq_workspace_bytes(n)
+
+
+def bitnet_w2a8_linear_seq(entries, workspace=None, stream=None):
+    """One kernel for a list of batch-1 decode linears.  entries: sequence of
+    (Weight, x, y, wait_for) with x fp32 [cols] and y fp32 [rows] CUDA tensors
+    (or views) and wait_for -1 or the index of the entry whose y x reads.
+    workspace: uint8 CUDA tensor of bitnet_w2a8_linear_seq_workspace_bytes(n)
+    bytes, zero-filled before first use (needed only when an entry waits)."""
+    n = len(entries)
+    arr = (bitnet_linear_desc * max(n, 1))()
+    for i, (w, x, y, wait_for) in enumerate(entries):
+        arr[i].w = ctypes.pointer(w.struct)
+        arr[i].x_dev = _dptr(x, "float32", w.cols, f"x[{i}]")
+        arr[i].y_dev = _dptr(y, "float32", w.rows, f"y[{i}]")
+        arr[i].wait_for = int(wait_for)
+    ws = _dptr(workspace, "uint8", bitnet_w2a8_linear_seq_workspace_bytes(n), "workspace") if workspace is not None \
+        else None
+    _check(_lib.bitnet_w2a8_linear_seq(arr, n, ws, workspace.numel() if workspace is not None else 0,
+                                       _stream(stream)), "bitnet_w2a8_linear_seq")
 
 
 def bitnet_get_device_error(stream=None) -> int:

@@ -357,6 +357,69 @@ bitnet_status bitnet_w2a8_gemv_lut(const bitnet_weight *w, const int8_t *q_dev, 
     return e == cudaSuccess ? BITNET_OK : cuda_fail(e, "gemv_lut launch");
 }
 
+size_t bitnet_w2a8_linear_seq_workspace_bytes(int32_t n) {
+    return n >= 1 && n <= kSeqMaxLinears ? seq_workspace_bytes(n) : 0;
+}
+
+bitnet_status bitnet_w2a8_linear_seq(const bitnet_linear_desc *list, int32_t n, void *workspace_dev,
+                                     size_t workspace_bytes, bitnet_stream_t stream) {
+    t_detail[0] = 0;
+    if (!list) return fail(BITNET_ERR_NULL, "list is NULL");
+    if (n < 1 || n > kSeqMaxLinears) return fail(BITNET_ERR_SHAPE, "n=%d outside 1..%d", n, kSeqMaxLinears);
+    static thread_local SeqLinear sl[kSeqMaxLinears];
+    static thread_local uint64_t anc[kSeqMaxLinears][kSeqMaxLinears / 64];  // anc[i] bit m: m precedes i
+    bool any_wait = false;
+    for (int i = 0; i < n; i++) {
+        const bitnet_linear_desc &d = list[i];
+        bitnet_status s = check_weight(d.w);
+        if (s != BITNET_OK) return s;
+        if (!(d.w->flags & BITNET_WEIGHT_UNIFORM_ROWS) || d.w->cols > kSeqMaxK)
+            return fail(BITNET_ERR_UNSUPPORTED, "entry %d: the sequence kernel takes uniform rows and cols <= %d", i,
+                        kSeqMaxK);
+        if (!d.x_dev || !d.y_dev) return fail(BITNET_ERR_NULL, "entry %d: NULL x or y", i);
+        if (!aligned(d.x_dev, 16) || !aligned(d.y_dev, 4))
+            return fail(BITNET_ERR_ALIGN, "entry %d: x needs 16-byte, y 4-byte alignment", i);
+        if (d.wait_for < -1 || d.wait_for >= i)
+            return fail(BITNET_ERR_VALUE, "entry %d: wait_for %d must be -1 or a lower index", i, d.wait_for);
+        sl[i] = SeqLinear{d.w->data, d.w->rows, d.w->cols, d.x_dev, d.y_dev, d.wait_for};
+        for (int k = 0; k < kSeqMaxLinears / 64; k++) anc[i][k] = 0;
+        if (d.wait_for >= 0) {
+            const int j = d.wait_for;
+            for (int k = 0; k < kSeqMaxLinears / 64; k++) anc[i][k] = anc[j][k];
+            anc[i][j >> 6] |= 1ull << (j & 63);
+            any_wait = true;
+        }
+    }
+    // Hazards: y ranges disjoint; x of m may overlap y of i only if one of the
+    // two precedes the other through waits.
+    auto precedes = [&](int a, int b) { return (anc[b][a >> 6] >> (a & 63)) & 1ull; };
+    auto overlap = [](const void *p, size_t pn, const void *q, size_t qn) {
+        const uintptr_t a = (uintptr_t)p, b = (uintptr_t)q;
+        return a < b + qn && b < a + pn;
+    };
+    for (int i = 0; i < n; i++) {
+        const size_t yi = (size_t)sl[i].rows * 4;
+        for (int m = 0; m < n; m++) {
+            if (m != i && m < i && overlap(sl[i].y, yi, sl[m].y, (size_t)sl[m].rows * 4))
+                return fail(BITNET_ERR_VALUE, "entries %d and %d: y ranges overlap", m, i);
+            if (overlap(sl[m].x, (size_t)sl[m].cols * 4, sl[i].y, yi) && !(m != i && (precedes(i, m) || precedes(m, i))))
+                return fail(BITNET_ERR_VALUE, "entry %d reads x where entry %d writes y without a wait between them", m,
+                            i);
+        }
+    }
+    if (any_wait) {
+        if (!workspace_dev) return fail(BITNET_ERR_NULL, "entries wait for others: workspace is NULL");
+        if (!aligned(workspace_dev, 4)) return fail(BITNET_ERR_ALIGN, "workspace needs 4-byte alignment");
+        if (workspace_bytes < seq_workspace_bytes(n))
+            return fail(BITNET_ERR_BUFSIZE, "workspace %zu < %zu bytes", workspace_bytes, seq_workspace_bytes(n));
+    }
+    DeviceGlobals g;
+    cudaError_t e = device_globals(&g);
+    if (e != cudaSuccess) return cuda_fail(e, "device globals");
+    e = launch_decode_seq(sl, n, any_wait ? workspace_dev : nullptr, g, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? BITNET_OK : cuda_fail(e, "linear_seq launch");
+}
+
 static bitnet_status gemm_impl(const bitnet_weight *w, const int8_t *q_dev, const float *s_dev,
                                int64_t T, float *y_dev, int32_t *acc_dev, bitnet_stream_t stream) {
     t_detail[0] = 0;

@@ -93,6 +93,21 @@ cudaError_t launch_decode_lut(const void *data, int64_t rows, int64_t cols, cons
 int absmean_num_partials(int64_t n);
 cudaError_t launch_ternarize(const float *w, int64_t rows, int64_t cols, bool per_block, uint32_t *codes,
                              float *scales, double *partials, float *gamma_slot, cudaStream_t st);
+// One linear of a sequence call (decode_seq.cu): repacked weight data with
+// uniform rows, fp32 x [cols], fp32 y [rows], and the index of the linear whose
+// y this x reads (-1: x is ready at launch).
+constexpr int kSeqMaxLinears = 256;
+constexpr int kSeqMaxK = 16384;
+struct SeqLinear {
+    const void *data;
+    int64_t rows, cols;
+    const float *x;
+    float *y;
+    int dep;
+};
+size_t seq_workspace_bytes(int n);
+cudaError_t launch_decode_seq(const SeqLinear *list, int n, void *workspace, const DeviceGlobals &g,
+                              cudaStream_t st);
 cudaError_t launch_gemm(const void *data, int64_t rows, int64_t cols, bool uniform,
                         const int8_t *q, const float *s, int64_t T, float *y, int32_t *acc,
                         const DeviceGlobals &g, cudaStream_t st);

@@ -84,35 +84,6 @@ struct DecArgs {
     int B;         // tokens (batched kernel)
 };
 
-// Shared-memory word of activation word m (bytes 4m .. 4m+3 of q): lane-part t
-// of block j, slot 2*group + half, so that lane t's words qa0 qb0 qa1 qb1 qa2
-// qb2 qa3 qb3 of a block are contiguous.
-__device__ __forceinline__ int perm_word(int m) {
-    const int w = m & 31;
-    return (m & ~31) | ((w & 3) << 3) | ((w >> 3) << 1) | ((w >> 2) & 1);
-}
-
-// Exact int -> fp32 for |v| < 2^22 with one integer add and one fp32 add:
-// the bits 0x4B400000 + v encode 1.5 * 2^23 + v.
-__device__ __forceinline__ float int_to_float(int v) {
-    return __fsub_rn(__int_as_float(0x4B400000 + v), 12582912.0f);
-}
-
-// The activation quantiser's q = rint(x * s) (one fp32 multiply, ties to
-// even) for four activations of a row with |x| <= absmax: then
-// |x * s| <= 127 * (1 + 2^-24)^2 < 127.5, so q lies in [-127, 127] and the
-// clamp never acts for finite x.  Adding 1.5 * 2^23 (round-to-nearest-even)
-// leaves rint(v) in the low mantissa bits, and the low byte of those bits is q
-// as an int8; three byte permutes pack the four bytes.  (NaN or Inf in x give
-// unspecified bytes here.)
-__device__ __forceinline__ uint32_t quant4_fast(float4 v, float s) {
-    const uint32_t b0 = __float_as_uint(__fadd_rn(__fmul_rn(v.x, s), 12582912.0f));
-    const uint32_t b1 = __float_as_uint(__fadd_rn(__fmul_rn(v.y, s), 12582912.0f));
-    const uint32_t b2 = __float_as_uint(__fadd_rn(__fmul_rn(v.z, s), 12582912.0f));
-    const uint32_t b3 = __float_as_uint(__fadd_rn(__fmul_rn(v.w, s), 12582912.0f));
-    return __byte_perm(__byte_perm(b0, b1, 0x0040), __byte_perm(b2, b3, 0x0040), 0x5410);
-}
-
 // One warp's share of a CTA's (row tile, block) items and the ring of
 // shared-memory slots its tiles move through.  Items run in memory order:
 // item i is row tile i / nb, block i % nb, 512-byte tile (r0 * nb + i).

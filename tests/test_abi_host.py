@@ -142,3 +142,48 @@ def test_device_calls_validate_before_touching_the_gpu(b):
     w2.bytes = 1 << 20
     w2.data = 128
     assert lib.bitnet_repack_device(16, 16, 16, 128, ctypes.byref(w2), None) == b.BITNET_ERR_ALIGN
+
+
+def test_linear_seq_validates_before_touching_the_gpu(b):
+    """bitnet_w2a8_linear_seq rejects, on the host: bad counts, waits on later
+    entries, overlapping outputs, reads of another entry's output without a
+    wait between them, weights without uniform rows, wide K, and a missing or
+    short workspace when an entry waits."""
+    lib = b.library()
+    W = b.bitnet_weight
+
+    def weight(rows, cols, flags=b.BITNET_WEIGHT_UNIFORM_ROWS):
+        w = W()
+        w.data, w.rows, w.cols, w.bytes = 256, rows, cols, 1 << 30
+        w.layout_version, w.flags = b.BITNET_LAYOUT_VERSION, flags
+        return w
+
+    keep = []
+
+    def call(entries, ws=None, wsb=0):
+        arr = (b.bitnet_linear_desc * max(len(entries), 1))()
+        for i, (w, x, y, d) in enumerate(entries):
+            keep.append(w)
+            arr[i].w = ctypes.pointer(w)
+            arr[i].x_dev, arr[i].y_dev, arr[i].wait_for = x, y, d
+        return lib.bitnet_w2a8_linear_seq(arr, len(entries), ws, wsb, None)
+
+    A = 1 << 20  # fake device addresses, never dereferenced on the host
+    w1, w2 = weight(64, 256), weight(32, 128)
+    assert lib.bitnet_w2a8_linear_seq(None, 1, None, 0, None) == b.BITNET_ERR_NULL
+    assert call([]) == b.BITNET_ERR_SHAPE
+    assert lib.bitnet_w2a8_linear_seq_workspace_bytes(0) == 0
+    assert lib.bitnet_w2a8_linear_seq_workspace_bytes(3) >= 16
+    assert call([(w1, A, A + 4096, 0)]) == b.BITNET_ERR_VALUE                      # waits on itself
+    assert call([(w1, A, A + 4096, -2)]) == b.BITNET_ERR_VALUE
+    assert call([(w1, A, A + 4096, -1), (w2, A + 8192, A + 4096 + 128, -1)]) == b.BITNET_ERR_VALUE  # y overlap
+    assert call([(w1, A, A + 4096, -1), (w2, A + 4096, A + 8192, -1)]) == b.BITNET_ERR_VALUE  # x reads y, no wait
+    assert call([(w1, A, A, -1)]) == b.BITNET_ERR_VALUE                              # reads its own output
+    assert call([(w1, A + 4, A + 4096, -1)]) == b.BITNET_ERR_ALIGN
+    assert call([(w1, None, A + 4096, -1)]) == b.BITNET_ERR_NULL
+    assert call([(weight(64, 256, flags=0), A, A + 4096, -1)]) == b.BITNET_ERR_UNSUPPORTED
+    assert call([(weight(64, 16384 + 128), A, A + (1 << 22), -1)]) == b.BITNET_ERR_UNSUPPORTED
+    chain = [(w1, A, A + 4096, -1), (w2, A + 4096, A + 8192, 0)]
+    assert call(chain) == b.BITNET_ERR_NULL                                           # waits need a workspace
+    assert call(chain, A + 65536, 4) == b.BITNET_ERR_BUFSIZE
+    assert call(chain, A + 65538, 1 << 12) == b.BITNET_ERR_ALIGN
