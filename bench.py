@@ -189,120 +189,128 @@ class ClockSampler:
 
 # ----------------------------------------------------------- our arm --
 
-def build_weights(b, torch, dev, layers, shapes, seed_base):
-    """Seeded fp32 N(0,1) weights drawn on the device, ternarised (per-tensor
-    absmean) and packed by the library, then repacked.  Untimed setup."""
+def build_weights(b, torch, dev, layers, shapes, config):
+    """Seeded fp32 N(0,1) weights (the splitmix64 + Box-Muller stream of
+    synthetic/, drawn on the device), ternarised with per-tensor absmean and
+    packed by the library, then repacked.  Untimed setup."""
+    import synthetic as syn
     ws = {}
     maxn = max(o * k for _, o, k in shapes)
     maxo, maxk = max(o for _, o, _ in shapes), max(k for _, _, k in shapes)
-    wbuf = torch.empty(maxn, dtype=torch.float32, device=dev)
     cbuf = torch.empty(maxn // 4, dtype=torch.uint8, device=dev)
     sbuf = torch.empty(maxn // 128, dtype=torch.float32, device=dev)
     wsp = torch.empty(b.bitnet_ternarize_workspace_bytes(maxo, maxk) + 4096, dtype=torch.uint8, device=dev)
-    gen = torch.Generator(device=dev)
     for l in range(layers):
         for m, (name, o, k) in enumerate(shapes):
-            gen.manual_seed(seed_base ^ (l << 24) ^ (m << 16) ^ 1)
-            w = wbuf[:o * k]
-            w.normal_(generator=gen)
+            w = syn.normal_device(syn.seed_for(config, l, m, syn.KIND_WEIGHT), o * k, dev)
             b.bitnet_ternarize_absmean_device(w, o, k, b.BITNET_ABSMEAN_PER_TENSOR, cbuf[:o * k // 4],
                                               sbuf[:o * k // 128], wsp)
             data = torch.empty(b.bitnet_repacked_bytes(o, k), dtype=torch.uint8, device=dev)
             ws[(l, name)] = b.bitnet_repack_device(cbuf[:o * k // 4], sbuf[:o * k // 128], o, k, data)
-    del wbuf, cbuf, sbuf, wsp
+            del w
+    del cbuf, sbuf, wsp
     return ws
 
 
-def make_inputs(torch, dev, layers, shapes, B, seed_base, outliers=True):
-    """x for every linear, one flat fp32 buffer (device) + pinned host copy."""
-    total = sum(B * k for _, _, k in shapes) * layers
-    gen = torch.Generator(device="cpu")
-    gen.manual_seed(seed_base ^ 2)
-    host = torch.randn(total, generator=gen, dtype=torch.float32)
-    views, off = {}, 0
+def make_inputs(torch, dev, layers, shapes, B, config, outliers=True):
+    """x for every linear from the host recipe of synthetic/ (N(0,1), a fixed
+    1% of channels x20): one flat fp32 device buffer and its pinned host copy."""
+    import numpy as np
+
+    import synthetic as syn
+    parts, views, off = [], {}, 0
     for l in range(layers):
         for m, (name, o, k) in enumerate(shapes):
-            x = host[off:off + B * k].view(B, k)
-            if outliers:
-                g2 = torch.Generator(device="cpu")
-                g2.manual_seed(seed_base ^ (m << 16) ^ 3)
-                ch = torch.randperm(k, generator=g2)[: k // 100]
-                x[:, ch] *= 20.0
+            parts.append(syn.activations(syn.seed_for(config, l, m, syn.KIND_ACT), B, k, outliers=outliers,
+                                         outlier_seed=syn.seed_for(config, 0, m, syn.KIND_OUTLIER)).reshape(-1))
             views[(l, name)] = (off, B * k)
             off += B * k
-    pinned = host.pin_memory()
-    return pinned, pinned.to(dev), views
+    host = torch.from_numpy(np.concatenate(parts)).pin_memory()
+    return host, host.to(dev), views
+
+
+class Timer:
+    """CUDA-graph replays timed with CUDA events on the replay stream."""
+
+    def __init__(self, torch, stream, dev):
+        self.torch, self.stream, self.dev = torch, stream, dev
+
+    def capture(self, fn, warm=2):
+        t = self.torch
+        with t.cuda.stream(self.stream):
+            for _ in range(warm):
+                fn()
+        t.cuda.synchronize(self.dev)
+        g = t.cuda.CUDAGraph()
+        with t.cuda.graph(g, stream=self.stream):
+            fn()
+        return g
+
+    def ms(self, graph, replays=20, passes=5, pre=None):
+        """Median over `passes` of the mean ms per replay (`pre` runs untimed
+        before each pass, e.g. an L2 flush)."""
+        t = self.torch
+        out = []
+        for _ in range(passes):
+            with t.cuda.stream(self.stream):
+                if pre:
+                    pre()
+                e0, e1 = t.cuda.Event(enable_timing=True), t.cuda.Event(enable_timing=True)
+                e0.record(self.stream)
+                for _ in range(replays):
+                    graph.replay()
+                e1.record(self.stream)
+            e1.synchronize()
+            out.append(e0.elapsed_time(e1) / replays)
+        return sorted(out)[len(out) // 2]
+
+
+def hbm(nbytes, ms, peak):
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return {"us": round(ms * 1e3, 3), "GB/s": round(gbs, 1), "frac": round(gbs / peak, 4)}
+
+
+def linear_entries(weights, layers, shapes, x_dev, xviews, ys, chain=False):
+    """(Weight, x, y, wait_for) for the sequence call: every linear with its own
+    x, or (chain) each x the first K outputs of the previous linear's y."""
+    ents = []
+    for l in range(layers):
+        for name, o, k in shapes:
+            i = len(ents)
+            key = (l, name)
+            if chain and i > 0:
+                ents.append((weights[key], ys[i - 1][:k], ys[i], i - 1))
+            else:
+                xo, xn = xviews[key]
+                ents.append((weights[key], x_dev[xo:xo + xn], ys[i], -1))
+    return ents
 
 
 def run_ours(args, rank, world, dev):
-    import numpy as np
     import torch
 
     import ternary_weight_absmax_b200 as b
 
     torch.cuda.set_device(dev)
     B = 1
-    seed = 0xB17E7 ^ (CONFIG_ID << 40)
-    weights = build_weights(b, torch, dev, LAYERS, SHAPES, seed)
-    x_host, x_dev, xviews = make_inputs(torch, dev, LAYERS, SHAPES, B, seed)
-    qbuf = {key: torch.empty(B * k, dtype=torch.int8, device=dev)
-            for key in weights for (n, _, k) in SHAPES if n == key[1]}
-    sbuf = {key: torch.empty(B, dtype=torch.float32, device=dev) for key in weights}
+    peaks = read_peaks()
+    peak = peaks["hbm_gbs"]
+    weights = build_weights(b, torch, dev, LAYERS, SHAPES, CONFIG_ID)
+    x_host, x_dev, xviews = make_inputs(torch, dev, LAYERS, SHAPES, B, CONFIG_ID)
     ytot = sum(B * o for _, o, _ in SHAPES) * LAYERS
     y_dev = torch.empty(ytot, dtype=torch.float32, device=dev)
     y_host = torch.empty(ytot, dtype=torch.float32).pin_memory()
-    yviews, off = {}, 0
+    ys, off = [], 0
     for l in range(LAYERS):
         for name, o, k in SHAPES:
-            yviews[(l, name)] = y_dev[off:off + B * o]
+            ys.append(y_dev[off:off + B * o])
             off += B * o
-
+    n_lin = LAYERS * len(SHAPES)
     stream = torch.cuda.Stream(device=dev)
-    launches_per_step = 0
-
-    def step(gemv_only=False, only=None):
-        """Two C-ABI calls per linear: bitnet_quant_act, bitnet_w2a8_gemv."""
-        n = 0
-        for l in range(LAYERS):
-            for name, o, k in SHAPES:
-                if only is not None and name != only:
-                    continue
-                key = (l, name)
-                xo, xn = xviews[key]
-                if not gemv_only:
-                    b.bitnet_quant_act(x_dev[xo:xo + xn], B, k, qbuf[key], sbuf[key])
-                    n += 1
-                b.bitnet_w2a8_gemv(weights[key], qbuf[key], sbuf[key], B, yviews[key])
-                n += 1
-        return n
-
-    def fused_step():
-        """One C-ABI call per linear: bitnet_w2a8_linear (quantise + GEMV)."""
-        n = 0
-        for l in range(LAYERS):
-            for name, o, k in SHAPES:
-                key = (l, name)
-                xo, xn = xviews[key]
-                b.bitnet_w2a8_linear(weights[key], x_dev[xo:xo + xn], B, yviews[key])
-                n += 1
-        return n
-
-    # Warm the quantised inputs once so GEMV-only graphs read real q, s.
-    with torch.cuda.stream(stream):
-        step()
-    torch.cuda.synchronize(dev)
-
-    def capture(fn):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream):
-            cnt = fn()
-        return g, cnt
-
-    g_step, launches_per_step = capture(fused_step)
-    g_two, two_launches = capture(lambda: step())
-    g_gemv, gemv_launches = capture(lambda: step(gemv_only=True))
-    g_shape = {name: capture(lambda name=name: step(gemv_only=True, only=name))[0] for name, _, _ in SHAPES}
-    flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    T = Timer(torch, stream, dev)
+    seq = linear_entries(weights, LAYERS, SHAPES, x_dev, xviews, ys)
+    g_step = T.capture(lambda: b.bitnet_w2a8_linear_seq(seq))
+    launches_per_step = 1
 
     def barrier():
         if world > 1:
@@ -310,29 +318,13 @@ def run_ours(args, rank, world, dev):
             dist.barrier()
         torch.cuda.synchronize(dev)
 
-    def timed(graph, reps, pre=None):
-        """Device ms per replay, CUDA events on the replay stream."""
-        ms = []
-        for _ in range(reps):
-            if pre:
-                with torch.cuda.stream(stream):
-                    pre()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            with torch.cuda.stream(stream):
-                e0.record(stream)
-                graph.replay()
-                e1.record(stream)
-            e1.synchronize()
-            ms.append(e0.elapsed_time(e1))
-        return ms
-
     clocks = ClockSampler(dev)
     clocks.start()
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
             g_step.replay()
     barrier()
-    # ---- timed region: K steps back to back ----
+    # ---- timed region: K steps back to back (the 520 MB of weights exceed L2) ----
     clocks.mark("t0")
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
@@ -346,22 +338,7 @@ def run_ours(args, rank, world, dev):
     step_ms_local = e0.elapsed_time(e1) / args.steps
     clocks.stop()
 
-    # ---- the two-call path (bitnet_quant_act + bitnet_w2a8_gemv) ----
-    two_ms = timed(g_two, max(3, min(50, args.steps)))
-    two_ms_step = sorted(two_ms)[len(two_ms) // 2]
-    # ---- GEMV-only replays (roofline of the dominant kernel) ----
-    gemv_ms = timed(g_gemv, max(3, min(20, args.steps)))
-    gemv_ms_per_step = sorted(gemv_ms)[len(gemv_ms) // 2]
-    # ---- per-shape GEMV, L2 flushed before each pass ----
-    per_shape = {}
-    for name, o, k in SHAPES:
-        ms = timed(g_shape[name], 7, pre=lambda: flush.fill_(1.0))
-        med = sorted(ms)[len(ms) // 2] / LAYERS
-        per_shape[name] = {"out": o, "K": k, "us": round(med * 1e3, 3),
-                           "GB/s": round(gemv_bytes(o, k) / (med * 1e-3) / 1e9, 1)}
-    del flush
-
-    # ---- e2e: pinned host x -> device, the captured C-ABI calls, y -> host ----
+    # ---- e2e: pinned host x -> device, the C-ABI call, y -> pinned host ----
     def e2e_once():
         with torch.cuda.stream(stream):
             x_dev.copy_(x_host, non_blocking=True)
@@ -370,7 +347,7 @@ def run_ours(args, rank, world, dev):
     for _ in range(3):
         e2e_once()
     torch.cuda.synchronize(dev)
-    e2e_steps = max(3, min(args.steps, 200))
+    e2e_steps = max(3, min(args.steps, 500))
     f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
         f0.record(stream)
@@ -381,77 +358,221 @@ def run_ours(args, rank, world, dev):
     f1.synchronize()
     e2e_ms_local = f0.elapsed_time(f1) / e2e_steps
 
-    # ---- prefill GEMM (T=2048) ----
-    prefill = run_prefill(b, torch, dev, stream, seed)
-    small_batch = run_small_batch(b, torch, dev, stream, seed, weights)
-    lut = run_lut(b, torch, dev, stream, weights)
+    per_rank_bytes = fused_step_bytes()
+    side = {}
+    # ---- the same step, one bitnet_w2a8_linear call per linear ----
+    g_calls = T.capture(lambda: [b.bitnet_w2a8_linear(w, x, 1, y) for (w, x, y, _) in seq])
+    side["per_call_step"] = dict(hbm(per_rank_bytes, T.ms(g_calls, 20), peak), launches=n_lin,
+                                 how="bitnet_w2a8_linear per linear (batch-1 decode kernel, programmatic "
+                                     "dependent launch), 120 calls in one CUDA graph")
+    del g_calls
+    # ---- dependent chain: each x is the first K outputs of the previous y ----
+    chain = linear_entries(weights, LAYERS, SHAPES, x_dev, xviews, ys, chain=True)
+    work = torch.zeros(b.bitnet_w2a8_linear_seq_workspace_bytes(n_lin), dtype=torch.uint8, device=dev)
+    try:
+        g_chain = T.capture(lambda: b.bitnet_w2a8_linear_seq(chain, work))
+        g_chain_calls = T.capture(lambda: [b.bitnet_w2a8_linear(w, x, 1, y) for (w, x, y, _) in chain])
+        side["chained_step"] = {
+            "seq": dict(hbm(per_rank_bytes, T.ms(g_chain, 20), peak), launches=1),
+            "per_call": dict(hbm(per_rank_bytes, T.ms(g_chain_calls, 20), peak), launches=n_lin),
+            "how": "linear i reads the first K outputs of linear i-1 (QKV->O->gate+up->down->next QKV): one "
+                   "bitnet_w2a8_linear_seq call whose entries wait for their producer on the device, vs one "
+                   "bitnet_w2a8_linear call per linear"}
+        del g_chain, g_chain_calls
+    except Exception as e:  # reported beside the headline, never instead of it
+        side["chained_step"] = {"error": f"{type(e).__name__}: {e}"}
+    del g_step
+    torch.cuda.synchronize(dev)
+    side["per_shape"] = run_per_shape(b, torch, dev, T, weights, peak)
+    side["llama8b_sweep"] = run_llama8b(b, torch, dev, T, peaks)
+    side["prefill"] = run_prefill(b, torch, dev, T, peaks)
+    side["small_batch_gemv"] = run_small_batch(b, torch, dev, T, weights, peak)
+    side["block_scale"] = run_block_scale(b, torch, dev, T, peaks)
+    side["lut_gemv_b1"] = run_lut(b, torch, dev, T, weights)
 
     status = b.bitnet_get_device_error(stream.cuda_stream)
     if status != b.BITNET_OK:
         raise RuntimeError(f"device error after bench: {b.bitnet_status_string(status)}")
 
-    gbytes, qbytes = step_bytes()
-    per_rank_bytes = fused_step_bytes()
-    step_ms, e2e_ms, gemv_ms_max, two_ms_max = reduce_max(
-        [step_ms_local, e2e_ms_local, gemv_ms_per_step, two_ms_step], dev)
+    step_ms, e2e_ms = reduce_max([step_ms_local, e2e_ms_local], dev)
     value, _ = aggregate([step_ms] * world, [per_rank_bytes] * world)
     e2e_value, _ = aggregate([e2e_ms] * world, [per_rank_bytes] * world)
-
-    peaks = read_peaks()
-    # Dominant kernel: the batch-1 decode kernel behind bitnet_w2a8_linear, one
-    # launch per linear of the step; its average launch time is the step time
-    # (CUDA events on the launch stream, timed region above) over the launches.
+    # Dominant kernel: decode_seq_kernel, one launch per step; its average
+    # launch time is the step time (CUDA events on the launch stream, timed
+    # region above).
     launch_us = step_ms * 1e3 / launches_per_step
     bytes_per_launch = per_rank_bytes / launches_per_step
     achieved = bytes_per_launch / (launch_us * 1e-6) / 1e9
-    roofline = {"kernel": "decode_b1_kernel (bitnet_w2a8_linear, batch 1, uniform rows)", "bound": "hbm",
-                "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": round(achieved / peaks["hbm_gbs"], 4), "peak_source": peaks["source"],
-                "traffic": read_traffic(), "bytes_per_launch": round(bytes_per_launch, 1),
+    traffic, traffic_note = read_traffic("decode_seq_kernel", bytes_per_launch)
+    roofline = {"kernel": "decode_seq_kernel (bitnet_w2a8_linear_seq, 120 batch-1 linears per launch)",
+                "bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(achieved / peak, 4), "peak_source": peaks["source"], "traffic": traffic,
+                "traffic_source": traffic_note, "bytes_per_launch": round(bytes_per_launch, 1),
                 "launch_us": round(launch_us, 3)}
 
     out = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_ms, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
-        "data": "synthetic (seeded N(0,1) weights ternarised on device; N(0,1) activations, 1% channels x20)",
-        "path": "bitnet_w2a8_linear per linear (activation quantisation fused into the GEMV)",
+        "data": "synthetic (splitmix64 + Box-Muller N(0,1) weights, per-tensor absmean ternary; N(0,1) "
+                "activations with 1% of channels x20)",
+        "path": "bitnet_w2a8_linear_seq: one call per step over the 120 linears, each quantising its own "
+                "fp32 x (absmax int8) and computing its fp32 y",
         "config": {"workload": WORKLOAD, "shapes_out_x_K": [[o, k] for _, o, k in SHAPES], "layers": LAYERS,
-                   "batch": B, "linears_per_step": LAYERS * len(SHAPES),
-                   "l2": "inputs larger than L2 (520 MB packed weights per step); per-shape passes flush L2",
-                   "graph": "the 120 C-ABI calls of a step captured in one CUDA graph",
+                   "batch": B, "linears_per_step": n_lin,
+                   "inputs": "every linear has its own seeded input (the linears of the step do not depend on "
+                             "each other); chained_step reports the dependent variant",
+                   "l2": "inputs larger than L2 (520 MB packed weights per step, read once per step)",
+                   "graph": "the step's C-ABI call captured in a CUDA graph and replayed",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
-        "per_shape_gemv": per_shape,
-        "two_call_step": {"ms_per_step": round(two_ms_max, 4),
-                          "GB/s": round(aggregate([two_ms_max] * world, [gbytes + qbytes] * world)[0], 2),
-                          "launches_per_step": two_launches,
-                          "how": "bitnet_quant_act + bitnet_w2a8_gemv per linear, same graph replay timing"},
-        "gemv_only_ms_per_step": round(gemv_ms_max, 4),
-        "prefill": prefill,
-        "small_batch_gemv": small_batch,
-        "lut_gemv_b1": lut,
+        **side,
         "roofline": roofline,
         "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "ms_per_step": round(e2e_ms, 4),
                 "h2d_bytes_per_step": int(x_host.numel() * 4), "d2h_bytes_per_step": int(y_host.numel() * 4),
-                "how": "pinned x copied in, graph of the step's C-ABI calls, y copied out, per step"},
+                "how": "pinned x copied in, the step's C-ABI call (graph), y copied out, per step"},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks.summary(),
     }
     return out
 
 
+def run_per_shape(b, torch, dev, T, weights, peak):
+    """Per shape of the step: (a) one bitnet_w2a8_linear call (latency of an
+    isolated launch: 30 calls on the 30 layers' weights in a graph, each with
+    its own cold x, L2 flushed before each pass), (b) sustained: the 30 layers'
+    weights of that shape in one bitnet_w2a8_linear_seq call."""
+    res = {}
+    try:
+        flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+        for m, (name, o, k) in enumerate(SHAPES):
+            ws = [weights[(l, name)] for l in range(LAYERS)]
+            xs = [torch.randn(k, device=dev) for _ in range(LAYERS)]
+            ys = [torch.empty(o, device=dev) for _ in range(LAYERS)]
+            g1 = T.capture(lambda: [b.bitnet_w2a8_linear(w, x, 1, y) for w, x, y in zip(ws, xs, ys)])
+            g2 = T.capture(lambda: b.bitnet_w2a8_linear_seq([(w, x, y, -1) for w, x, y in zip(ws, xs, ys)]))
+            one = T.ms(g1, 1, 7, pre=lambda: flush.fill_(1.0)) / LAYERS
+            sus = T.ms(g2, 1, 7, pre=lambda: flush.fill_(1.0)) / LAYERS
+            nb = linear_bytes(o, k)
+            res[name] = {"out": o, "K": k, "bytes": nb, "per_call": hbm(nb, one, peak),
+                         "sustained_seq": hbm(nb, sus, peak)}
+            del g1, g2
+        del flush
+    except Exception as e:
+        res["error"] = f"{type(e).__name__}: {e}"
+    return res
+
+
+SHAPES_8B = [("qkv", 6144, 4096), ("o", 4096, 4096), ("gate_up", 28672, 4096), ("down", 4096, 14336)]
+LAYERS_8B = 32
+CONFIG_8B = 4
+
+
+def run_llama8b(b, torch, dev, T, peaks):
+    """Llama-3-8B-shaped ternary linears, 32 layers (1.97 GB packed): the
+    sustained-HBM sweep at batch 1 (independent inputs and the dependent
+    chain), at batch 16 and as prefill (T = 1024)."""
+    peak = peaks["hbm_gbs"]
+    res = {"shapes_out_x_K": [[o, k] for _, o, k in SHAPES_8B], "layers": LAYERS_8B}
+    try:
+        weights = build_weights(b, torch, dev, LAYERS_8B, SHAPES_8B, CONFIG_8B)
+        packed = sum(weights[key].rows * weights[key].cols // 4 for key in weights)
+        res["packed_bytes"] = packed
+        n_lin = LAYERS_8B * len(SHAPES_8B)
+        for B in (1, 16):
+            x_host, x_dev, xviews = make_inputs(torch, dev, LAYERS_8B, SHAPES_8B, B, CONFIG_8B)
+            ytot = sum(B * o for _, o, _ in SHAPES_8B) * LAYERS_8B
+            y_dev = torch.empty(ytot, dtype=torch.float32, device=dev)
+            ys, off = [], 0
+            for l in range(LAYERS_8B):
+                for name, o, k in SHAPES_8B:
+                    ys.append(y_dev[off:off + B * o])
+                    off += B * o
+            nbytes = fused_step_bytes(SHAPES_8B, LAYERS_8B, B)
+            if B == 1:
+                seq = linear_entries(weights, LAYERS_8B, SHAPES_8B, x_dev, xviews, ys)
+                g = T.capture(lambda: b.bitnet_w2a8_linear_seq(seq))
+                res["b1_seq"] = dict(hbm(nbytes, T.ms(g, 10), peak), launches=1)
+                del g
+                g = T.capture(lambda: [b.bitnet_w2a8_linear(w, x, 1, y) for (w, x, y, _) in seq])
+                res["b1_per_call"] = dict(hbm(nbytes, T.ms(g, 10), peak), launches=n_lin)
+                del g
+                chain = linear_entries(weights, LAYERS_8B, SHAPES_8B, x_dev, xviews, ys, chain=True)
+                work = torch.zeros(b.bitnet_w2a8_linear_seq_workspace_bytes(n_lin), dtype=torch.uint8, device=dev)
+                try:
+                    g = T.capture(lambda: b.bitnet_w2a8_linear_seq(chain, work))
+                    res["b1_chain_seq"] = dict(hbm(nbytes, T.ms(g, 10), peak), launches=1)
+                    del g
+                except Exception as e:
+                    res["b1_chain_seq"] = {"error": f"{type(e).__name__}: {e}"}
+            else:
+                ents = linear_entries(weights, LAYERS_8B, SHAPES_8B, x_dev, xviews, ys)
+                g = T.capture(lambda: [b.bitnet_w2a8_linear(w, x, B, y) for (w, x, y, _) in ents])
+                res[f"b{B}_per_call"] = dict(hbm(nbytes, T.ms(g, 5), peak), launches=n_lin,
+                                             how="bitnet_w2a8_linear per linear (activation quantisation and "
+                                                 "the batched GEMV)")
+                del g
+            del x_host, x_dev, y_dev, ys
+        # Prefill T = 1024: act-quant + GEMM per shape (layer 0's weights).
+        res["prefill_T1024"] = prefill_shapes(b, torch, dev, T, peaks, [(n, o, k, weights[(0, n)])
+                                                                        for n, o, k in SHAPES_8B], 1024)
+        del weights
+        torch.cuda.empty_cache()
+    except Exception as e:
+        res["error"] = f"{type(e).__name__}: {e}"
+    return res
+
+
+def prefill_shapes(b, torch, dev, T, peaks, cases, tokens):
+    out = {}
+    for name, o, k, w in cases:
+        x = torch.randn(tokens * k, dtype=torch.float32, device=dev)
+        q = torch.empty(tokens * k, dtype=torch.int8, device=dev)
+        s = torch.empty(tokens, dtype=torch.float32, device=dev)
+        y = torch.empty(tokens * o, dtype=torch.float32, device=dev)
+        g_q = T.capture(lambda: b.bitnet_quant_act(x, tokens, k, q, s))
+        g_m = T.capture(lambda: b.bitnet_w2a8_gemm(w, q, s, tokens, y))
+        g_b = T.capture(lambda: (b.bitnet_quant_act(x, tokens, k, q, s), b.bitnet_w2a8_gemm(w, q, s, tokens, y)))
+        mq, mm, mb = T.ms(g_q, 10), T.ms(g_m, 10), T.ms(g_b, 10)
+        ops = 2.0 * tokens * o * k
+        tops = ops / (mm * 1e-3) / 1e12
+        qbytes = 4 * tokens * k + tokens * k + 4 * tokens
+        out[name] = {"out": o, "K": k, "T": tokens, "gemm_us": round(mm * 1e3, 2), "TOPS": round(tops, 1),
+                     "frac_of_int8_peak": round(tops / peaks["int8_tops"], 4),
+                     "act_quant_us": round(mq * 1e3, 2),
+                     "act_quant_GB/s": round(qbytes / (mq * 1e-3) / 1e9, 1),
+                     "linear_us": round(mb * 1e3, 2)}
+        del g_q, g_m, g_b
+    return out
+
+
+def run_prefill(b, torch, dev, T, peaks):
+    res = {"int8_peak_TOPS": peaks["int8_tops"], "peak_source": peaks["int8_source"]}
+    try:
+        weights = build_weights(b, torch, dev, 1, PREFILL, 3)
+        for tokens in (512, 2048):
+            res[f"T{tokens}"] = prefill_shapes(b, torch, dev, T, peaks,
+                                               [(n, o, k, weights[(0, n)]) for n, o, k in PREFILL], tokens)
+        best = max(v["TOPS"] for tt in ("T512", "T2048") for v in res[tt].values())
+        res["best_frac_of_int8_peak"] = round(best / peaks["int8_tops"], 4)
+        del weights
+    except Exception as e:  # reported beside the headline, never instead of it
+        res["error"] = f"{type(e).__name__}: {e}"
+    return res
+
+
 SMALL_BATCH = [("o", 2560, 2560), ("gate_up", 13824, 2560), ("wide", 20480, 3200)]
 SMALL_BATCH_B = (1, 4, 16)
 
 
-def run_small_batch(b, torch, dev, stream, seed, weights):
+def run_small_batch(b, torch, dev, T, weights, peak):
     """bitnet_w2a8_gemv at B = 1, 4, 16 on the standalone shapes: one call per
     distinct weight copy (30 copies of the step's O and gate+up weights, 12
-    copies of 20480 x 3200), L2 flushed with a 512 MB write before each timed
-    pass; median of 5 passes, us per call and algorithmic GB/s."""
+    copies of 20480 x 3200), one q shared by the calls, L2 flushed with a
+    512 MB write before each timed pass; median of 5 passes, us per call and
+    algorithmic GB/s."""
     res = {}
     try:
-        wide = build_weights(b, torch, dev, 12, [("wide", 20480, 3200)], seed ^ 0x99)
+        wide = build_weights(b, torch, dev, 12, [("wide", 20480, 3200)], 2)
         flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
         for name, o, k in SMALL_BATCH:
             ws = [wide[(l, name)] for l in range(12)] if name == "wide" else \
@@ -462,29 +583,10 @@ def run_small_batch(b, torch, dev, stream, seed, weights):
                 q = torch.empty(B * k, dtype=torch.int8, device=dev)
                 s = torch.empty(B, dtype=torch.float32, device=dev)
                 y = torch.empty(B * o, dtype=torch.float32, device=dev)
-                with torch.cuda.stream(stream):
-                    b.bitnet_quant_act(x, B, k, q, s)
-                    for w in ws:
-                        b.bitnet_w2a8_gemv(w, q, s, B, y)
-                torch.cuda.synchronize(dev)
-                g = torch.cuda.CUDAGraph()
-                with torch.cuda.graph(g, stream=stream):
-                    for w in ws:
-                        b.bitnet_w2a8_gemv(w, q, s, B, y)
-                ms = []
-                for _ in range(5):
-                    with torch.cuda.stream(stream):
-                        flush.fill_(1.0)
-                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                    with torch.cuda.stream(stream):
-                        e0.record(stream)
-                        g.replay()
-                        e1.record(stream)
-                    e1.synchronize()
-                    ms.append(e0.elapsed_time(e1) / len(ws))
-                med = sorted(ms)[len(ms) // 2]
-                res[name][f"B{B}"] = {"us": round(med * 1e3, 3),
-                                      "GB/s": round(gemv_bytes(o, k, B) / (med * 1e-3) / 1e9, 1)}
+                b.bitnet_quant_act(x, B, k, q, s)
+                g = T.capture(lambda: [b.bitnet_w2a8_gemv(w, q, s, B, y) for w in ws])
+                ms = T.ms(g, 1, 5, pre=lambda: flush.fill_(1.0)) / len(ws)
+                res[name][f"B{B}"] = hbm(gemv_bytes(o, k, B), ms, peak)
                 del g
         del flush, wide
     except Exception as e:  # reported beside the headline, never instead of it
@@ -492,7 +594,46 @@ def run_small_batch(b, torch, dev, stream, seed, weights):
     return res
 
 
-def run_lut(b, torch, dev, stream, weights):
+def run_block_scale(b, torch, dev, T, peaks):
+    """The general (per-block scale) paths on varied scales: every 128-weight
+    block with its own absmean scale (the library's per-block ternariser).
+    GEMV B = 1 (general kernel, fp64 epilogue) over 30 copies of 13824 x 2560
+    with L2 flushed, and the GEMM at T = 2048 (block-scale tcgen05 path)."""
+    res = {}
+    try:
+        import synthetic as syn
+        o, k = 13824, 2560
+        cbuf = torch.empty(o * k // 4, dtype=torch.uint8, device=dev)
+        sbuf = torch.empty(o * k // 128, dtype=torch.float32, device=dev)
+        wsp = torch.empty(b.bitnet_ternarize_workspace_bytes(o, k) + 4096, dtype=torch.uint8, device=dev)
+        ws = []
+        for l in range(30):
+            w = syn.normal_device(syn.seed_for(5, l, 0, syn.KIND_WEIGHT), o * k, dev)
+            b.bitnet_ternarize_absmean_device(w, o, k, b.BITNET_ABSMEAN_PER_BLOCK, cbuf, sbuf, wsp)
+            data = torch.empty(b.bitnet_repacked_bytes(o, k), dtype=torch.uint8, device=dev)
+            ws.append(b.bitnet_repack_device(cbuf, sbuf, o, k, data))
+            assert not ws[-1].uniform
+        flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+        x = torch.randn(k, device=dev)
+        q = torch.empty(k, dtype=torch.int8, device=dev)
+        s = torch.empty(1, device=dev)
+        y = torch.empty(o, device=dev)
+        b.bitnet_quant_act(x, 1, k, q, s)
+        g = T.capture(lambda: [b.bitnet_w2a8_gemv(w, q, s, 1, y) for w in ws])
+        ms = T.ms(g, 1, 5, pre=lambda: flush.fill_(1.0)) / len(ws)
+        nb = o * k // 4 + o * k // 32 + k + 4 + 4 * o
+        res["gemv_b1_13824x2560"] = dict(hbm(nb, ms, peaks["hbm_gbs"]), bytes=nb,
+                                         how="bitnet_w2a8_gemv, general kernel (block scales, fp64 epilogue)")
+        del g, flush
+        res["gemm_T2048_13824x2560"] = prefill_shapes(b, torch, dev, T, peaks, [("gate_up", o, k, ws[0])], 2048)[
+            "gate_up"]
+        del ws, cbuf, sbuf, wsp
+    except Exception as e:
+        res["error"] = f"{type(e).__name__}: {e}"
+    return res
+
+
+def run_lut(b, torch, dev, T, weights):
     """The table-lookup GEMV variant against the dp4a GEMV at batch 1 on the
     step's four shapes: 30 calls on the 30 layers' weights, one q, L2 flushed
     before each timed pass, median of 5 passes, us per call."""
@@ -505,89 +646,15 @@ def run_lut(b, torch, dev, stream, weights):
             q = torch.empty(k, dtype=torch.int8, device=dev)
             s = torch.empty(1, dtype=torch.float32, device=dev)
             y = torch.empty(o, dtype=torch.float32, device=dev)
-            calls = {"lut": lambda w: b.bitnet_w2a8_gemv_lut(w, q, s, y),
-                     "dp4a": lambda w: b.bitnet_w2a8_gemv(w, q, s, 1, y)}
+            b.bitnet_quant_act(x, 1, k, q, s)
             res[name] = {"out": o, "K": k}
-            for kind, call in calls.items():
-                with torch.cuda.stream(stream):
-                    b.bitnet_quant_act(x, 1, k, q, s)
-                    for w in ws:
-                        call(w)
-                torch.cuda.synchronize(dev)
-                g = torch.cuda.CUDAGraph()
-                with torch.cuda.graph(g, stream=stream):
-                    for w in ws:
-                        call(w)
-                ms = []
-                for _ in range(5):
-                    with torch.cuda.stream(stream):
-                        flush.fill_(1.0)
-                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                    with torch.cuda.stream(stream):
-                        e0.record(stream)
-                        g.replay()
-                        e1.record(stream)
-                    e1.synchronize()
-                    ms.append(e0.elapsed_time(e1) / len(ws))
-                res[name][f"{kind}_us"] = round(sorted(ms)[2] * 1e3, 3)
+            for kind, call in (("lut", lambda w: b.bitnet_w2a8_gemv_lut(w, q, s, y)),
+                               ("dp4a", lambda w: b.bitnet_w2a8_gemv(w, q, s, 1, y))):
+                g = T.capture(lambda: [call(w) for w in ws])
+                res[name][f"{kind}_us"] = round(T.ms(g, 1, 5, pre=lambda: flush.fill_(1.0)) / len(ws) * 1e3, 3)
                 del g
         del flush
     except Exception as e:  # reported beside the headline, never instead of it
-        res["error"] = f"{type(e).__name__}: {e}"
-    return res
-
-
-def run_prefill(b, torch, dev, stream, seed):
-    res = {"T": PREFILL_T, "shapes": {}}
-    try:
-        weights = build_weights(b, torch, dev, 1, PREFILL, seed ^ 0x77)
-        for name, o, k in PREFILL:
-            w = weights[(0, name)]
-            T = PREFILL_T
-            x = torch.randn(T * k, dtype=torch.float32, device=dev)
-            q = torch.empty(T * k, dtype=torch.int8, device=dev)
-            s = torch.empty(T, dtype=torch.float32, device=dev)
-            y = torch.empty(T * o, dtype=torch.float32, device=dev)
-            with torch.cuda.stream(stream):
-                b.bitnet_quant_act(x, T, k, q, s)
-                for _ in range(3):
-                    b.bitnet_w2a8_gemm(w, q, s, T, y)
-            torch.cuda.synchronize(dev)
-            g = torch.cuda.CUDAGraph()
-            reps = 10
-            with torch.cuda.graph(g, stream=stream):
-                for _ in range(reps):
-                    b.bitnet_w2a8_gemm(w, q, s, T, y)
-            ms = []
-            for _ in range(5):
-                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                with torch.cuda.stream(stream):
-                    e0.record(stream)
-                    g.replay()
-                    e1.record(stream)
-                e1.synchronize()
-                ms.append(e0.elapsed_time(e1) / reps)
-            med = sorted(ms)[len(ms) // 2]
-            ops = 2.0 * T * o * k
-            aq = []
-            for _ in range(5):
-                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                with torch.cuda.stream(stream):
-                    e0.record(stream)
-                    b.bitnet_quant_act(x, T, k, q, s)
-                    e1.record(stream)
-                e1.synchronize()
-                aq.append(e0.elapsed_time(e1))
-            res["shapes"][name] = {"out": o, "K": k, "gemm_us": round(med * 1e3, 2),
-                                   "TOPS": round(ops / (med * 1e-3) / 1e12, 1),
-                                   "act_quant_us": round(sorted(aq)[2] * 1e3, 2)}
-            del g
-        peaks = read_peaks()
-        best = max(v["TOPS"] for v in res["shapes"].values())
-        res["int8_peak_TOPS"] = peaks["int8_tops"]
-        res["frac_of_int8_peak"] = round(best / peaks["int8_tops"], 4)
-        res["peak_source"] = peaks["int8_source"]
-    except Exception as e:  # the prefill figure is reported beside the headline, never instead of it
         res["error"] = f"{type(e).__name__}: {e}"
     return res
 
@@ -597,24 +664,41 @@ def read_peaks():
     try:
         with open(p) as f:
             d = json.load(f)
-        hbm, bf16 = float(d["hbm_gbs"]), float(d["bf16_tflops"])
+        hbm_, bf16 = float(d["hbm_gbs"]), float(d["bf16_tflops"])
         src = "measured (MEASURED_PEAKS.json: copy bandwidth)"
         isrc = "measured bf16 cuBLAS burst x 2 (nominal int8:bf16 dense ratio)"
     except (OSError, KeyError, ValueError):
-        hbm, bf16 = 6650.0, 1590.0
-        src = isrc = "fallback (6.65 TB/s, 1.59 PFLOP/s bf16)"
-    return {"hbm_gbs": hbm, "int8_tops": 2.0 * bf16, "source": src, "int8_source": isrc}
+        hbm_, bf16 = 6650.0, 1590.0
+        src = isrc = "fallback (6.65 TB/s, 1.59 PFLOP/s bf16; no MEASURED_PEAKS.json)"
+    return {"hbm_gbs": hbm_, "int8_tops": 2.0 * bf16, "source": src, "int8_source": isrc}
 
 
-def read_traffic():
-    """DRAM bytes per decode-kernel launch (mean over the step's four shapes)
-    from the committed ncu summary, if present."""
-    p = os.path.join(ROOT, "profiles", "decode_traffic.json")
+def source_digest(*names):
+    import hashlib
+    h = hashlib.sha256()
+    for n in names:
+        with open(os.path.join(ROOT, "ternary_weight_absmax_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def read_traffic(kernel, bytes_per_launch):
+    """DRAM bytes (read + write) per launch of `kernel` from the committed ncu
+    summary, scaled to this launch's algorithmic bytes when the capture ran a
+    smaller case; null if the kernel's source changed since the capture."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(p) as f:
-            return json.load(f).get("bytes_per_launch")
-    except (OSError, ValueError):
-        return None
+            d = json.load(f)[kernel]
+    except (OSError, ValueError, KeyError):
+        return None, "no ncu capture on record"
+    if d.get("source_digest") != source_digest(*d.get("sources", [])):
+        return None, "kernel changed since the ncu capture"
+    ratio = bytes_per_launch / d["algorithmic_bytes"]
+    note = f"ncu dram__bytes_read.sum + dram__bytes_write.sum, {d['case']}"
+    if abs(ratio - 1.0) > 1e-6:
+        note += f", scaled x{ratio:.4f} to this launch's algorithmic bytes"
+    return round(d["dram_bytes"] * ratio), note
 
 
 # ----------------------------------------------------- reference arm --
@@ -678,38 +762,85 @@ def run_reference(args, rank, world):
     return out
 
 
-def cpu_baseline(seconds=12.0):
-    """The oracle timed on one host core on a bounded sample of the workload:
-    layer 0's four linears, all output rows, batch 1, repeated for ~12 s."""
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def cpu_baseline(seconds=8.0):
+    """The oracle (plain single-threaded C) timed on the host on a bounded
+    sample of the workload: layer 0's four linears (all rows, batch 1), (a) on
+    one core, (b) split by output rows over one thread per host core (the C
+    call releases the GIL), each for about `seconds`; plus the prefill GEMM
+    oracle on a 64-token slice of 13824 x 2560, all cores, extrapolated
+    linearly to T = 2048."""
+    import concurrent.futures as cf
+
     import numpy as np
 
     import oracle
     import synthetic as syn
 
     oracle.build()
-    B = 1
+    cores = os.cpu_count() or 1
     cases = []
     for m, (name, o, k) in enumerate(SHAPES):
         w = syn.normal_matrix(syn.seed_for(CONFIG_ID, 0, m, syn.KIND_WEIGHT), o, k)
         t, g = oracle.absmean_tensor(w)
         codes = oracle.pack_i2s(t)
         sc = np.full((o, k // 128), g, dtype=np.float32)
-        x = syn.activations(syn.seed_for(CONFIG_ID, 0, m, syn.KIND_ACT), B, k, outliers=True)
+        x = syn.activations(syn.seed_for(CONFIG_ID, 0, m, syn.KIND_ACT), 1, k, outliers=True)
         cases.append((o, k, codes, sc, x))
     per_layer = sum(linear_bytes(o, k) for o, k, *_ in cases)
-    t0 = time.perf_counter()
-    n = 0
-    while True:
+
+    def layer(pool=None):
         for o, k, codes, sc, x in cases:
             q, s, _ = oracle.quant_act(x)
-            oracle.linear(codes, sc, k, q, s)
-        n += 1
-        dt = time.perf_counter() - t0
-        if dt >= seconds:
-            break
-    return {"value": round(per_layer * n / dt / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "sample": f"layer 0 of the 30 (4 linears, all rows, batch 1), {n} passes in {dt:.1f} s",
-            "us_per_layer": round(dt / n * 1e6, 1)}
+            if pool is None:
+                oracle.linear(codes, sc, k, q, s)
+            else:
+                step = (o + cores - 1) // cores
+                list(pool.map(lambda r0: oracle.linear(codes[r0:r0 + step], sc[r0:r0 + step], k, q, s),
+                              range(0, o, step)))
+
+    def timed(pool=None):
+        t0 = time.perf_counter()
+        n = 0
+        while True:
+            layer(pool)
+            n += 1
+            dt = time.perf_counter() - t0
+            if dt >= seconds:
+                return n, dt
+
+    n1, dt1 = timed()
+    with cf.ThreadPoolExecutor(max_workers=cores) as pool:
+        nN, dtN = timed(pool)
+        # GEMM oracle: 64 tokens of 13824 x 2560, rows split over the cores.
+        o, k, codes, sc, _ = cases[2]
+        x = syn.activations(syn.seed_for(3, 0, 0, syn.KIND_ACT), 64, k)
+        q, s, _ = oracle.quant_act(x)
+        step = (o + cores - 1) // cores
+        t0 = time.perf_counter()
+        list(pool.map(lambda r0: oracle.linear(codes[r0:r0 + step], sc[r0:r0 + step], k, q, s), range(0, o, step)))
+        dtg = time.perf_counter() - t0
+    gemm_tops = 2.0 * 64 * o * k / dtg / 1e12
+    return {"value": round(per_layer * n1 / dt1 / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"layer 0 of the 30 (4 linears, all rows, batch 1), {n1} passes in {dt1:.1f} s on one core",
+            "us_per_layer": round(dt1 / n1 * 1e6, 1),
+            "all_cores": {"value": round(per_layer * nN / dtN / 1e9, 4), "unit": "GB/s", "cores": cores,
+                          "us_per_layer": round(dtN / nN * 1e6, 1),
+                          "sample": f"same layer, output rows split over {cores} threads, {nN} passes in {dtN:.1f} s"},
+            "gemm_T2048_13824x2560_extrapolated": {
+                "TOPS": round(gemm_tops, 6), "ms": round(dtg * 2048 / 64 * 1e3, 1), "cores": cores,
+                "sample": "64 tokens timed on all cores, scaled linearly to T = 2048 (extrapolated)"},
+            "cpu_model": cpu_model(), "nproc": cores}
 
 
 # ------------------------------------------------------- small cases --

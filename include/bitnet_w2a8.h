@@ -209,18 +209,24 @@ bitnet_status bitnet_quant_act(const float *x_dev, int64_t T, int64_t K, int8_t 
  * The linear layer (async).
  * ---------------------------------------------------------------------- */
 
-/* Decode / small-batch GEMV, 1 <= B <= 16:
+/* Decode / small-batch GEMV, 1 <= B <= 64:
  *   y[b][o] = (sum_j scale[o][j] * acc[b][o][j]) / s[b]
  * with acc the int32 block dot products of the ternary weights and q.
  * q_dev: B*K int8 (16-byte aligned); s_dev: B fp32; y_dev: B*rows fp32
- * (4-byte aligned).  The int32 sums are exact.  The sum over blocks runs in
- * fp64 and is rounded once to fp32, except on weights with uniform rows
- * (BITNET_WEIGHT_UNIFORM_ROWS, the per-tensor absmean case) and K <= 16384,
- * the decode calls: there y = scale * acc * (1/s) in fp32 (three roundings,
- * within 2.4e-7 relative of the fp64 value).
- * Errors: NULL, SHAPE (B outside 1..16, K mismatch), ALIGN, VALUE (w not
- * repacked), CUDA.  The decode kernels wait (bounded) on their weight copies;
- * a wait that runs out latches BITNET_ERR_TIMEOUT.
+ * (4-byte aligned).  The int32 sums are exact.  Kernels and epilogues:
+ *   - weights with uniform rows (BITNET_WEIGHT_UNIFORM_ROWS, the per-tensor
+ *     absmean case): y = scale * acc * (1/s) in fp32 (three roundings, within
+ *     2.4e-7 relative of the fp64 value), bit for bit the same for every B:
+ *     B = 1 and K <= 16384 the batch-1 decode kernel (dp4a); B = 2, 3 and
+ *     K <= 16384 the batched decode kernel (dp4a); B >= 4 the tensor-core
+ *     kernel (tcgen05 int8 MMA, weights on the M side, K split over a thread
+ *     block cluster); otherwise the general kernel;
+ *   - other weights: the sum over blocks runs in fp64 and is rounded once
+ *     (the general kernel, exact for B <= 16; the GEMM's block-scale path,
+ *     y = fp32(sum * (1/s)), for B > 16).
+ * Errors: NULL, SHAPE (B outside 1..64, K mismatch), ALIGN, VALUE (w not
+ * repacked), CUDA.  Bounded device waits that run out latch
+ * BITNET_ERR_TIMEOUT.
  * The GEMV, the fused linear and the quantiser use programmatic dependent
  * launch: a GEMV may start reading its (constant) weights while the kernel
  * before it on the stream is still running, and reads q, s (or x) and writes
@@ -229,16 +235,21 @@ bitnet_status bitnet_quant_act(const float *x_dev, int64_t T, int64_t K, int8_t 
 bitnet_status bitnet_w2a8_gemv(const bitnet_weight *w, const int8_t *q_dev, const float *s_dev,
                                int64_t B, float *y_dev, bitnet_stream_t stream);
 
-/* Decode linear layer in one kernel, 1 <= B <= 16: quantises fp32 x [B][K]
- * exactly as bitnet_quant_act does, then computes what bitnet_w2a8_gemv
- * computes, without a global round trip of q (every CTA re-quantises x into
- * shared memory).  x_dev: B*K fp32 (16-byte aligned); y_dev: B*rows fp32.
- * q_out_dev (B*K int8) and s_out_dev (B fp32) are optional (NULL = not
- * written; 4-byte aligned) and receive the quantised activations.  The fp32
- * epilogue is the GEMV's at B = 1 on uniform rows with K <= 16384; at
- * B >= 2 this call runs the general kernel (fp64 epilogue).
- * Errors: NULL, SHAPE, ALIGN, VALUE, BUFSIZE, CUDA; BITNET_ERR_TIMEOUT is
- * latched as for the GEMV. */
+/* Decode linear layer, 1 <= B <= 64: quantises fp32 x [B][K] exactly as
+ * bitnet_quant_act does, then computes what bitnet_w2a8_gemv computes.
+ * x_dev: B*K fp32 (16-byte aligned); y_dev: B*rows fp32.  q_out_dev (B*K
+ * int8) and s_out_dev (B fp32) are optional at B <= 16 (NULL = not written)
+ * and receive the quantised activations.
+ *   - Without q_out_dev / s_out_dev (B <= 16): ONE kernel; every CTA
+ *     re-quantises x into shared memory, no global round trip of q.  B = 1 on
+ *     uniform rows with K <= 16384 is the batch-1 decode kernel (fp32
+ *     epilogue); otherwise the general kernel (fp64 epilogue).
+ *   - With both (required for B > 16; q_out_dev then 16-byte aligned): the
+ *     quantiser writes them, and the GEMV of bitnet_w2a8_gemv reads them (two
+ *     kernels, the second overlapping its weight fetch with the first): the
+ *     tensor-core kernel for uniform rows from B = 4 on.
+ * Errors: NULL (B > 16 without q_out_dev / s_out_dev), SHAPE, ALIGN, VALUE,
+ * BUFSIZE, CUDA; BITNET_ERR_TIMEOUT is latched as for the GEMV. */
 bitnet_status bitnet_w2a8_linear(const bitnet_weight *w, const float *x_dev, int64_t B, float *y_dev,
                                  int8_t *q_out_dev, float *s_out_dev, bitnet_stream_t stream);
 

@@ -120,3 +120,41 @@ def integer_rows(seed: int, T: int, K: int, peak: int = 127) -> np.ndarray:
     sign = np.where((pick >> np.uint64(32)) & np.uint64(1), -1, 1)
     x[np.arange(T), col] = sign * peak
     return x.astype(np.float32)
+
+
+def _as_i64(v: int) -> int:
+    """The two's-complement int64 with the same 64 bits as the uint64 v."""
+    v &= 2**64 - 1
+    return v - 2**64 if v >= 2**63 else v
+
+
+def normal_device(seed: int, n: int, device, chunk: int = 1 << 24):
+    """The same N(0,1) stream as normal_f32(seed, n), drawn with torch on
+    `device` (for the benchmark's multi-gigabyte weight sets).  splitmix64 runs
+    in int64 (wrapping multiply; right shifts masked to be logical); the
+    Box-Muller step runs in fp64 with torch's log/cos/sin, so an element may
+    differ from the host stream in its last fp32 bit."""
+    import torch
+    out = torch.empty(n, dtype=torch.float32, device=device)
+    g, m1, m2 = _as_i64(int(GOLDEN)), _as_i64(int(M1)), _as_i64(int(M2))
+
+    def lsr(z, k):
+        return (z >> k) & ((1 << (64 - k)) - 1)
+
+    def mix(cnt):
+        z = cnt.add(1).mul_(g).add_(_as_i64(seed))
+        z = (z ^ lsr(z, 30)).mul_(m1)
+        z = (z ^ lsr(z, 27)).mul_(m2)
+        return z ^ lsr(z, 31)
+
+    for p0 in range(0, (n + 1) // 2, chunk):
+        p1 = min((n + 1) // 2, p0 + chunk)
+        pairs = torch.arange(p0, p1, dtype=torch.int64, device=device)
+        u1 = (lsr(mix(2 * pairs), 11).double() + 1.0) * 2.0**-53
+        u2 = lsr(mix(2 * pairs + 1), 11).double() * 2.0**-53
+        r = torch.sqrt(-2.0 * torch.log(u1))
+        th = 2.0 * torch.pi * u2
+        pair_out = torch.stack((r * torch.cos(th), r * torch.sin(th)), dim=1).reshape(-1).float()
+        lo, hi = 2 * p0, min(n, 2 * p1)
+        out[lo:hi] = pair_out[: hi - lo]
+    return out

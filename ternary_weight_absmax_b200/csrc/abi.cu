@@ -281,20 +281,33 @@ bitnet_status bitnet_quant_act(const float *x_dev, int64_t T, int64_t K, int8_t 
     return e == cudaSuccess ? BITNET_OK : cuda_fail(e, "quant_act launch");
 }
 
+// Device work of a GEMV on given q, s: the tensor-core kernel for uniform
+// rows from kTcMinBatch tokens, the decode / general kernels up to 16 tokens,
+// the GEMM's block-scale path (per-block fp64 sums) beyond.
+static cudaError_t gemv_dispatch(const bitnet_weight *w, const int8_t *q_dev, const float *s_dev, int64_t B,
+                                 float *y_dev, int32_t *acc_dev, const DeviceGlobals &g, cudaStream_t st) {
+    const bool uniform = (w->flags & BITNET_WEIGHT_UNIFORM_ROWS) != 0;
+    if (uniform && !acc_dev && B >= kTcMinBatch && gemv_tc_supported(w->rows, w->cols, B))
+        return launch_gemv_tc(w->data, w->rows, w->cols, q_dev, s_dev, B, y_dev, g, st);
+    if (B <= 16)
+        return launch_gemv(w->data, w->rows, w->cols, uniform, q_dev, s_dev, B, y_dev, acc_dev, nullptr, nullptr,
+                           nullptr, g, st);
+    return launch_gemm(w->data, w->rows, w->cols, false, q_dev, s_dev, B, y_dev, acc_dev, g, st);
+}
+
 static bitnet_status gemv_impl(const bitnet_weight *w, const int8_t *q_dev, const float *s_dev,
                                int64_t B, float *y_dev, int32_t *acc_dev, bitnet_stream_t stream) {
     t_detail[0] = 0;
     bitnet_status s = check_weight(w);
     if (s != BITNET_OK) return s;
-    if (B < 1 || B > 16) return fail(BITNET_ERR_SHAPE, "GEMV batch %lld outside 1..16", (long long)B);
+    if (B < 1 || B > 64) return fail(BITNET_ERR_SHAPE, "GEMV batch %lld outside 1..64", (long long)B);
     if (!q_dev || !s_dev || !y_dev) return fail(BITNET_ERR_NULL, "NULL pointer");
     if (!aligned(q_dev, 16) || !aligned(s_dev, 4) || !aligned(y_dev, 4) || (acc_dev && !aligned(acc_dev, 4)))
         return fail(BITNET_ERR_ALIGN, "q needs 16-byte, s/y/acc 4-byte alignment");
     DeviceGlobals g;
     cudaError_t e = device_globals(&g);
     if (e != cudaSuccess) return cuda_fail(e, "device globals");
-    e = launch_gemv(w->data, w->rows, w->cols, (w->flags & BITNET_WEIGHT_UNIFORM_ROWS) != 0, q_dev, s_dev, B,
-                    y_dev, acc_dev, nullptr, nullptr, nullptr, g, reinterpret_cast<cudaStream_t>(stream));
+    e = gemv_dispatch(w, q_dev, s_dev, B, y_dev, acc_dev, g, reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? BITNET_OK : cuda_fail(e, "gemv launch");
 }
 
@@ -303,16 +316,29 @@ static bitnet_status linear_impl(const bitnet_weight *w, const float *x_dev, int
     t_detail[0] = 0;
     bitnet_status s = check_weight(w);
     if (s != BITNET_OK) return s;
-    if (B < 1 || B > 16) return fail(BITNET_ERR_SHAPE, "linear batch %lld outside 1..16", (long long)B);
+    if (B < 1 || B > 64) return fail(BITNET_ERR_SHAPE, "linear batch %lld outside 1..64", (long long)B);
     if (!x_dev || !y_dev) return fail(BITNET_ERR_NULL, "NULL pointer");
-    if (!aligned(x_dev, 16) || !aligned(y_dev, 4) || (q_out_dev && !aligned(q_out_dev, 4)) ||
+    const bool staged = B >= 2 && q_out_dev && s_out_dev;
+    if (B > 16 && !staged)
+        return fail(BITNET_ERR_NULL, "linear batch %lld > 16 needs q_out and s_out", (long long)B);
+    if (!aligned(x_dev, 16) || !aligned(y_dev, 4) || (q_out_dev && !aligned(q_out_dev, staged ? 16 : 4)) ||
         (s_out_dev && !aligned(s_out_dev, 4)) || (acc_dev && !aligned(acc_dev, 4)))
-        return fail(BITNET_ERR_ALIGN, "x needs 16-byte, y/q_out/s_out/acc 4-byte alignment");
+        return fail(BITNET_ERR_ALIGN, "x needs 16-byte, y/s_out/acc 4-byte, q_out 4-byte (16 from B = 2 "
+                                      "with s_out) alignment");
     DeviceGlobals g;
     cudaError_t e = device_globals(&g);
     if (e != cudaSuccess) return cuda_fail(e, "device globals");
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (staged) {
+        // Two kernels: the quantiser into the caller's q_out / s_out, then the
+        // GEMV on them (programmatic dependent launch overlaps the GEMV's
+        // weight fetch with the quantiser).
+        e = launch_quant_act(x_dev, B, w->cols, q_out_dev, s_out_dev, nullptr, st);
+        if (e == cudaSuccess) e = gemv_dispatch(w, q_out_dev, s_out_dev, B, y_dev, acc_dev, g, st);
+        return e == cudaSuccess ? BITNET_OK : cuda_fail(e, "linear launch");
+    }
     e = launch_gemv(w->data, w->rows, w->cols, (w->flags & BITNET_WEIGHT_UNIFORM_ROWS) != 0, nullptr, nullptr, B,
-                    y_dev, acc_dev, x_dev, q_out_dev, s_out_dev, g, reinterpret_cast<cudaStream_t>(stream));
+                    y_dev, acc_dev, x_dev, q_out_dev, s_out_dev, g, st);
     return e == cudaSuccess ? BITNET_OK : cuda_fail(e, "linear launch");
 }
 

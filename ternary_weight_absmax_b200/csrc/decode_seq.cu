@@ -40,8 +40,9 @@
 // linears pays one grid-wide hand-off per linear but never waits for weights.
 // Dependent waits need every CTA resident: such calls are cooperative
 // launches (one CTA per SM).  Every wait is bounded; on a timeout the kernel
-// latches the error word, stops, waits (bounded) for its copies in flight and
-// returns.  The last CTA to finish zeroes the counters for the next call.
+// latches the error word, raises an abort word that ends the other CTAs'
+// waits, stops, waits (bounded) for its copies in flight and returns.  The
+// last CTA to finish zeroes the counters and the abort word for the next call.
 #include <atomic>
 
 #include "common.cuh"
@@ -85,6 +86,7 @@ struct SeqLin {
 struct SeqArgs {
     unsigned *done;        // [n] tiles finished per linear (workspace), or null
     unsigned *exit_count;  // CTAs finished (workspace), or null
+    unsigned *abort;       // set by a CTA that gave up, so the others stop waiting (workspace), or null
     unsigned *err;
     const unsigned *wait_limit;
     int n, nwaves;
@@ -208,12 +210,18 @@ __global__ void __launch_bounds__(kThreads, 1) decode_seq_kernel(const __grid_co
 
         // ---- A: producer, x, absmax, q, sum(q)
         if (l.dep >= 0 && tid == 0) {
+            // Each poll is an L2 round trip: a sixteenth of the copy-wait
+            // iteration cap and the wall-clock cap bound the wait; another
+            // CTA's abort ends it at once.
             const unsigned need = (unsigned)a.lin[l.dep].ntr;
+            const uint32_t dlim = limit >> 4 ? limit >> 4 : 1u;
             uint32_t it = 0;
+            ptx::WaitClock clk;
             while (ld_acquire_gpu(a.done + l.dep) < need) {
-                if (++it >= limit) {
+                if (++it >= dlim || clk.expired(it) || *reinterpret_cast<volatile unsigned *>(a.abort)) {
                     *bad_w = 1;
                     atomicOr(a.err, kErrTimeout);
+                    atomicExch(a.abort, 1u);
                     break;
                 }
             }
@@ -311,6 +319,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_seq_kernel(const __grid_co
                     if (lane == 0 && !*bad_w) {
                         *bad_w = 1;
                         atomicOr(a.err, kErrTimeout);
+                        if (a.abort) atomicExch(a.abort, 1u);
                     }
                     ok = false;
                     break;
@@ -380,6 +389,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_seq_kernel(const __grid_co
             __threadfence();
             for (int L = 0; L < n; L++) a.done[L] = 0u;
             *a.exit_count = 0u;
+            *a.abort = 0u;
             __threadfence();
         }
     }
@@ -387,7 +397,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_seq_kernel(const __grid_co
 
 }  // namespace
 
-size_t seq_workspace_bytes(int n) { return align_up((size_t)(n + 1) * sizeof(unsigned), 256); }
+size_t seq_workspace_bytes(int n) { return align_up((size_t)(n + 2) * sizeof(unsigned), 256); }
 
 cudaError_t launch_decode_seq(const SeqLinear *list, int n, void *workspace, const DeviceGlobals &g,
                               cudaStream_t st) {
@@ -438,6 +448,7 @@ cudaError_t launch_decode_seq(const SeqLinear *list, int n, void *workspace, con
     unsigned *ws = static_cast<unsigned *>(workspace);
     a.done = any_dep ? ws : nullptr;
     a.exit_count = any_dep ? ws + n : nullptr;
+    a.abort = any_dep ? ws + n + 1 : nullptr;
 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)num_sms());

@@ -39,13 +39,40 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
         : "memory");
     return ok != 0u;
 }
+// Nanosecond global timer.
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+// Wall-clock cap of every bounded wait: a try_wait may suspend the thread for
+// a system-dependent time, so an iteration cap alone does not bound the time.
+constexpr uint64_t kWaitCapNs = 2000000000ull;
+
+// Tracks the wall-clock cap of one wait: checked every 64 tries.
+struct WaitClock {
+    uint64_t t0 = 0;
+    __device__ __forceinline__ bool expired(uint32_t i) {
+        if ((i & 63u) != 63u) return false;
+        const uint64_t t = globaltimer_ns();
+        if (t0 == 0) {
+            t0 = t;
+            return false;
+        }
+        return t - t0 > kWaitCapNs;
+    }
+};
+
 // Waits for the phase with the given parity to complete, at most `limit`
-// tries; gives up early once *abort is set.  Returns false if it gave up.
+// tries and about kWaitCapNs; gives up early once *abort is set.  Returns
+// false if it gave up.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint32_t limit,
                                           const volatile int *abort) {
+    WaitClock clk;
     for (uint32_t i = 0; i < limit; i++) {
         if (mbar_try_wait(bar, parity)) return true;
         if (abort && *abort) return false;
+        if (clk.expired(i)) return false;
     }
     return false;
 }
@@ -73,9 +100,11 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *m, 
 // time (a whole main loop) so they do not take issue slots from busy warps.
 __device__ __forceinline__ bool mbar_wait_sleep(uint32_t bar, uint32_t parity, uint32_t limit,
                                                 const volatile int *abort, unsigned ns) {
+    WaitClock clk;
     for (uint32_t i = 0; i < limit; i++) {
         if (mbar_try_wait(bar, parity)) return true;
         if (abort && *abort) return false;
+        if (clk.expired(i)) return false;
         __nanosleep(ns);
     }
     return false;
@@ -173,6 +202,62 @@ __device__ __forceinline__ void tmem_wait_ld() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// D[tmem] (+)= A[tmem] x B[smem desc], 8-bit x 8-bit -> int32 (A read from
+// tensor memory: lane m holds row m, K packed four per 32-bit column).
+__device__ __forceinline__ void mma_i8_ta(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// 16 lanes x 128 bits, repeated 8 times along the columns (32 columns):
+// thread i writes v[2r] to (lane base + i/4, column 4r + i%4) and v[2r+1] to
+// (lane base + 8 + i/4, the same column), r = 0..7.
+__device__ __forceinline__ void tmem_st_16x128b_x8(uint32_t taddr, const uint32_t (&v)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.16x128b.x8.b32 [%0], "
+        "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]),
+        "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+        : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() {
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// 32 lanes x 16 consecutive 32-bit columns (thread i: lane base + i).
+__device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&v)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+          "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+        : "r"(taddr));
+}
+
+// ---- thread-block clusters ----------------------------------------------------
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+// Address of the same shared-memory offset in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t saddr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ void red_add_cluster(uint32_t addr, int v) {
+    asm volatile("red.relaxed.cluster.shared::cluster.add.s32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
 // Shared-memory matrix descriptor for a K-major operand stored in the
 // 128-byte swizzle layout: 8-row x 128-byte atoms, atoms 1024 bytes apart.
 __device__ __forceinline__ uint64_t desc_k_sw128(uint32_t saddr) {
@@ -185,10 +270,10 @@ __device__ __forceinline__ uint64_t desc_k_sw128(uint32_t saddr) {
     return d;
 }
 
-// Instruction descriptor, kind::i8: s8 A, s8 B, s32 D, both K-major.
-__host__ __device__ constexpr uint32_t idesc_i8(int M, int N) {
+// Instruction descriptor, kind::i8: s8 (or u8) A, s8 B, s32 D, both K-major.
+__host__ __device__ constexpr uint32_t idesc_i8(int M, int N, bool a_signed = true) {
     return (2u << 4)                        // D format: s32
-           | (1u << 7)                      // A format: signed 8-bit
+           | ((a_signed ? 1u : 0u) << 7)    // A format: signed / unsigned 8-bit
            | (1u << 10)                     // B format: signed 8-bit
            | ((uint32_t)(N >> 3) << 17)     // N / 8
            | ((uint32_t)(M >> 4) << 24);    // M / 16

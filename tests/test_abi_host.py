@@ -108,7 +108,9 @@ def test_device_calls_validate_before_touching_the_gpu(b):
     assert lib.bitnet_w2a8_gemv(ctypes.byref(w), 16, 16, 1, 16, None) == b.BITNET_ERR_VALUE
     w.layout_version = b.BITNET_LAYOUT_VERSION
     assert lib.bitnet_w2a8_gemv(ctypes.byref(w), 16, 16, 0, 16, None) == b.BITNET_ERR_SHAPE
-    assert lib.bitnet_w2a8_gemv(ctypes.byref(w), 16, 16, 17, 16, None) == b.BITNET_ERR_SHAPE
+    assert lib.bitnet_w2a8_gemv(ctypes.byref(w), 16, 16, 65, 16, None) == b.BITNET_ERR_SHAPE
+    # a fused linear beyond 16 tokens needs q_out / s_out to stage the quantised activations
+    assert lib.bitnet_w2a8_linear(ctypes.byref(w), 16, 17, 16, None, None, None) == b.BITNET_ERR_NULL
     assert lib.bitnet_w2a8_gemv(ctypes.byref(w), 17, 16, 1, 16, None) == b.BITNET_ERR_ALIGN
     w.bytes = 10
     assert lib.bitnet_w2a8_gemv(ctypes.byref(w), 16, 16, 1, 16, None) == b.BITNET_ERR_BUFSIZE
