@@ -847,10 +847,12 @@ def cpu_baseline(seconds=8.0):
 
 def run_case(args):
     """One kernel on one shape, for profiling: `--case gemv` runs
-    bitnet_w2a8_gemv and `--case linear` bitnet_w2a8_linear (activation
-    quantisation fused) over `--copies` distinct weights (so the weights exceed
-    L2), `--case gemm` runs bitnet_w2a8_gemm on one weight; `--reps` passes,
-    plain launches (no graph).  Prints one JSON line with the median time."""
+    bitnet_w2a8_gemv (batch `--batch`), `--case linear` bitnet_w2a8_linear,
+    both over `--copies` distinct weights (so the weights exceed L2); `--case
+    gemm` runs bitnet_w2a8_gemm on one weight (`--tokens`); `--case quant`
+    bitnet_quant_act on `--tokens` rows; `--case seq` one bitnet_w2a8_linear_seq
+    call over `--copies` linears of the shape.  `--reps` passes, plain launches
+    (no graph).  Prints one JSON line with the median time."""
     import torch
 
     import ternary_weight_absmax_b200 as b
@@ -858,36 +860,44 @@ def run_case(args):
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
     o, k = args.rows, args.cols
-    seed = 0xB17E7 ^ 0x5A5A
-    vec = args.case in ("gemv", "linear")
+    vec = args.case in ("gemv", "linear", "seq")
     copies = args.copies if vec else 1
-    ws = build_weights(b, torch, dev, copies, [("w", o, k)], seed)
+    ws = build_weights(b, torch, dev, copies, [("w", o, k)], 6)
     T = args.batch if vec else args.tokens
     x = torch.randn(T * k, dtype=torch.float32, device=dev)
     q = torch.empty(T * k, dtype=torch.int8, device=dev)
     s = torch.empty(T, dtype=torch.float32, device=dev)
-    y = torch.empty(T * o, dtype=torch.float32, device=dev)
+    y = torch.empty(copies * T * o, dtype=torch.float32, device=dev)
     b.bitnet_quant_act(x, T, k, q, s)
-    if args.case == "linear":
-        def call(w, q_, s_, T_, y_):
-            b.bitnet_w2a8_linear(w, x, T_, y_)
+    if args.case == "seq":
+        ents = [(ws[(c, "w")], x[:k], y[c * o:(c + 1) * o], -1) for c in range(copies)]
+        calls = [lambda: b.bitnet_w2a8_linear_seq(ents)]
+    elif args.case == "linear":
+        calls = [lambda w=ws[(c, "w")]: b.bitnet_w2a8_linear(w, x, T, y[:T * o], q if T > 1 else None,
+                                                              s if T > 1 else None) for c in range(copies)]
+    elif args.case == "gemv":
+        calls = [lambda w=ws[(c, "w")]: b.bitnet_w2a8_gemv(w, q, s, T, y[:T * o]) for c in range(copies)]
+    elif args.case == "quant":
+        calls = [lambda: b.bitnet_quant_act(x, T, k, q, s)]
     else:
-        call = b.bitnet_w2a8_gemv if args.case == "gemv" else b.bitnet_w2a8_gemm
+        calls = [lambda: b.bitnet_w2a8_gemm(ws[(0, "w")], q, s, T, y[:T * o])]
     times = []
     for _ in range(args.reps):
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
-        for c in range(copies):
-            call(ws[(c, "w")], q, s, T, y)
+        for call in calls:
+            call()
         e1.record()
         e1.synchronize()
         times.append(e0.elapsed_time(e1) * 1e3 / copies)
     assert b.bitnet_get_device_error() == b.BITNET_OK
     med = sorted(times)[len(times) // 2]
-    out = {"case": args.case, "out": o, "K": k, "T": T, "copies": copies, "us_per_launch": round(med, 3)}
+    out = {"case": args.case, "out": o, "K": k, "T": T, "copies": copies, "us_per_linear": round(med, 3)}
     if vec:
         nbytes = gemv_bytes(o, k, T) if args.case == "gemv" else linear_bytes(o, k, T)
         out["GB/s"] = round(nbytes / (med * 1e-6) / 1e9, 1)
+    elif args.case == "quant":
+        out["GB/s"] = round(5.0 * T * k / (med * 1e-6) / 1e9, 1)
     else:
         out["TOPS"] = round(2.0 * T * o * k / (med * 1e-6) / 1e12, 1)
     print(json.dumps(out), flush=True)
@@ -898,11 +908,11 @@ def run_case(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--steps", type=int, default=20000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--case", choices=["gemv", "linear", "gemm"], help="profile one kernel on one shape")
+    ap.add_argument("--case", choices=["gemv", "linear", "gemm", "quant", "seq"], help="profile one kernel on one shape")
     ap.add_argument("--rows", type=int, default=13824)
     ap.add_argument("--cols", type=int, default=2560)
     ap.add_argument("--batch", type=int, default=1)

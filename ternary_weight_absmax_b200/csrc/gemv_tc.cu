@@ -46,20 +46,24 @@
 namespace bitnet {
 namespace {
 
-constexpr int kStages = 6;        // pipeline stages = tensor-memory A buffers
 constexpr int kThreads = 192;     // 6 warps
-constexpr int kTmemCols = 256;    // accumulator at [0, 64), A buffers at 64 + 32 * stage
-constexpr int kAcol = 64;
+constexpr int kTmemCols = 256;    // accumulator at [0, NT), A buffers after it, 32 columns per stage
 constexpr uint32_t kDrainLimit = 1u << 22;
 
+// NT tokens per CTA: 16, 32, 64 (GEMV; K may be split over a cluster) or 128
+// (prefill tiles; no split).
 template <int NT>
 struct TcCfg {
+    static constexpr int kStages = NT <= 64 ? 6 : 4;          // pipeline stages = tensor-memory A buffers
+    static constexpr int kAcol = NT <= 64 ? 64 : 128;         // first A-buffer column
+    static_assert(kAcol + 32 * kStages <= kTmemCols, "tensor-memory columns");
     static constexpr int kQBytes = NT * 128;                  // activations of one block, 128-byte rows
     static constexpr int kCodeBytes = 8 * kTileBytes;         // eight 16-row code tiles of one block
     static constexpr int kStageBytes = kQBytes + kCodeBytes;  // multiple of 1024
+    static constexpr bool kSplit = NT <= 64;                  // K may be split over a cluster
     static constexpr int kRedStride = NT + 1;                 // int32 per row of the cluster sum (+1: banks)
     static constexpr int kOffRed = kStages * kStageBytes;
-    static constexpr int kOffSq = kOffRed + 128 * kRedStride * 4;
+    static constexpr int kOffSq = kOffRed + (kSplit ? 128 * kRedStride * 4 : 0);
     static constexpr int kOffInv = kOffSq + NT * 4;
     static constexpr int kOffBar = kOffInv + NT * 4;
     // At least 80 KB so that no more than two CTAs share an SM: two hold all
@@ -113,7 +117,8 @@ template <int NT>
 __global__ void __launch_bounds__(kThreads, 2)
 gemv_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constant__ CUtensorMap map_q, const TcArgs a) {
     using C = TcCfg<NT>;
-    constexpr int S = kStages;
+    constexpr int S = C::kStages;
+    constexpr int kAcol = C::kAcol;
     extern __shared__ unsigned char smem_raw[];
     const uint32_t raw = ptx::smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
@@ -121,6 +126,8 @@ gemv_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constant_
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = a.splits > 1 ? ptx::cluster_rank() : 0u;
     const int mt = (int)(blockIdx.x / (unsigned)a.splits);
+    const int b0 = (int)blockIdx.y * NT;            // first token of this CTA
+    const int bt = min(NT, a.B - b0);               // its tokens
     const int j0 = (int)((int64_t)rank * a.nb / a.splits);
     const int nj = (int)((int64_t)(rank + 1) * a.nb / a.splits) - j0;
     const uint32_t bars = base + C::kOffBar;
@@ -153,14 +160,15 @@ gemv_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constant_
         ptx::tmem_alloc(ptx::smem_u32(tmem_slot), kTmemCols);
         ptx::tmem_relinquish();
     }
-    for (int i = threadIdx.x; i < 128 * C::kRedStride; i += kThreads) red[i] = 0;
+    if (C::kSplit)
+        for (int i = threadIdx.x; i < 128 * C::kRedStride; i += kThreads) red[i] = 0;
     for (int i = threadIdx.x; i < NT; i += kThreads) sq[i] = 0;
     ptx::tc_fence_before();
     __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     // The first CTA's sum buffer is zero before any CTA of the cluster adds to it.
-    if (a.splits > 1) ptx::cluster_sync();
+    if (C::kSplit && a.splits > 1) ptx::cluster_sync();
 
     auto give_up = [&]() {
         *abort_flag = 1;
@@ -193,7 +201,7 @@ gemv_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constant_
                     ptx::mbar_arrive_expect_tx(full(s), C::kCodeBytes + C::kQBytes);
                     ptx::tma_load_3d(base + s * C::kStageBytes + C::kQBytes, &map_c, full(s), 0, j0 + it, mt * 8);
                 }
-                ptx::tma_load_2d(base + s * C::kStageBytes, &map_q, full(s), 128 * (j0 + it), 0);
+                ptx::tma_load_2d(base + s * C::kStageBytes, &map_q, full(s), 128 * (j0 + it), b0);
                 issued = it + 1;
             }
             // Copies in flight (the last S stages issued) land before the CTA
@@ -234,7 +242,7 @@ gemv_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constant_
         const int d = threadIdx.x - 64;                 // 0..127
         constexpr int kPer = 128 / NT;                  // threads per token for sum(q)
         const int tok = d / kPer, part = d % kPer;
-        if (d < a.B) inv[d] = __frcp_rn(a.s[d]);
+        if (d < bt) inv[d] = __frcp_rn(a.s[b0 + d]);
         const int row = quarter * 32 + lane;
         const int64_t o = (int64_t)mt * 128 + row;
         const float rs = o < a.rows ? __ldg(a.rowscale + o) : 0.0f;
@@ -272,45 +280,46 @@ gemv_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constant_
         }
         atomicAdd(sq + tok, sqa);
         asm volatile("bar.sync 1, 128;" ::: "memory");  // sum(q) and 1/s complete (decoder warps only)
-        int p[NT];
+        // The accumulator, 16 token columns at a time (thread = row): sum t*q =
+        // sum c*q - sum q; then y (no split) or an add into the first CTA.
         if (ok && warp_wait<true>(accf, 0, limit, abort_flag)) {
             ptx::tc_fence_after();
-#pragma unroll
-            for (int c0 = 0; c0 < NT; c0 += 16) {
+            const uint32_t dst = C::kSplit && a.splits > 1
+                                     ? ptx::map_to_rank(ptx::smem_u32(red + row * C::kRedStride), 0)
+                                     : 0u;
+#pragma unroll 1
+            for (int c0 = 0; c0 < NT && c0 < bt; c0 += 16) {
                 uint32_t v[16];
                 ptx::tmem_ld_32x32b_x16(tmem + tlane + (uint32_t)c0, v);
                 ptx::tmem_wait_ld();
 #pragma unroll
-                for (int i = 0; i < 16; i++) p[c0 + i] = (int)v[i] - sq[c0 + i];
+                for (int i = 0; i < 16; i++) {
+                    const int b = c0 + i;
+                    if (b >= bt) break;
+                    const int val = (int)v[i] - sq[b];
+                    if (!C::kSplit || a.splits == 1) {
+                        if (o < a.rows)
+                            a.y[(int64_t)(b0 + b) * a.rows + o] = __fmul_rn(__fmul_rn(rs, (float)val), inv[b]);
+                    } else {
+                        ptx::red_add_cluster(dst + 4u * b, val);
+                    }
+                }
             }
-        } else {
-            if (ok && lane == 0) give_up();
-#pragma unroll
-            for (int i = 0; i < NT; i++) p[i] = 0;
-        }
-        if (a.splits == 1) {
-            if (o < a.rows) {
-#pragma unroll
-                for (int b = 0; b < NT; b++)
-                    if (b < a.B) a.y[(int64_t)b * a.rows + o] = __fmul_rn(__fmul_rn(rs, (float)p[b]), inv[b]);
-            }
-        } else {
-            const uint32_t dst = ptx::map_to_rank(ptx::smem_u32(red + row * C::kRedStride), 0);
-#pragma unroll
-            for (int b = 0; b < NT; b++)
-                if (b < a.B) ptx::red_add_cluster(dst + 4u * b, p[b]);
+        } else if (ok && lane == 0) {
+            give_up();
         }
     }
 
-    if (a.splits > 1) {
+    if (C::kSplit && a.splits > 1) {
         ptx::cluster_sync();  // every CTA's partial sums have landed in the first CTA
         if (rank == 0 && warp >= 2) {
             const int row = (warp & 3) * 32 + lane;
             const int64_t o = (int64_t)mt * 128 + row;
             if (o < a.rows) {
                 const float rs = __ldg(a.rowscale + o);
-                for (int b = 0; b < a.B; b++)
-                    a.y[(int64_t)b * a.rows + o] = __fmul_rn(__fmul_rn(rs, (float)red[row * C::kRedStride + b]), inv[b]);
+                for (int b = 0; b < bt; b++)
+                    a.y[(int64_t)(b0 + b) * a.rows + o] =
+                        __fmul_rn(__fmul_rn(rs, (float)red[row * C::kRedStride + b]), inv[b]);
             }
         }
     }
@@ -375,7 +384,7 @@ cudaError_t run_tc(const void *data, const Layout &L, const int8_t *q, TcArgs a,
     }
     const int64_t mtiles = (L.rows + 127) / 128;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(mtiles * a.splits));
+    cfg.gridDim = dim3((unsigned)(mtiles * a.splits), (unsigned)((a.B + NT - 1) / NT));
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = C::kSmem;
     cfg.stream = st;
@@ -396,6 +405,23 @@ cudaError_t run_tc(const void *data, const Layout &L, const int8_t *q, TcArgs a,
 bool gemv_tc_supported(int64_t rows, int64_t cols, int64_t B) {
     (void)rows;
     return B >= 1 && B <= 64 && cols >= kQK && cols <= (int64_t(1) << 17);
+}
+
+cudaError_t launch_gemm_tc(const void *data, int64_t rows, int64_t cols, const int8_t *q, const float *s,
+                           int64_t T, float *y, const DeviceGlobals &g, cudaStream_t st) {
+    const Layout L = layout_of(rows, cols);
+    const unsigned char *base = static_cast<const unsigned char *>(data);
+    TcArgs a;
+    a.rowscale = reinterpret_cast<const float *>(base + L.off_rowscale);
+    a.s = s;
+    a.y = y;
+    a.err = g.err;
+    a.wait_limit = g.wait_limit;
+    a.rows = rows;
+    a.B = (int)T;
+    a.nb = (int)L.nb;
+    a.splits = 1;
+    return run_tc<128>(data, L, q, a, st);
 }
 
 cudaError_t launch_gemv_tc(const void *data, int64_t rows, int64_t cols, const int8_t *q, const float *s,

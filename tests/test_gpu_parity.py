@@ -25,7 +25,8 @@ def _need_cuda():
 
 @pytest.mark.parametrize("T,K,outliers", [(1, 128, False), (1, 512, False), (1, 2560, True), (33, 2560, True),
                                           (4, 6912, True), (2, 14336, False), (7, 3200, True),
-                                          (300, 1024, True)])
+                                          (300, 1024, True), (3, 32768, True), (2, 32896, True),
+                                          (1, 65536, False), (5, 384, True), (17, 4096, False)])
 def test_quant_act_bit_exact(T, K, outliers):
     x = syn.activations(syn.seed_for(0, T, K % 997, syn.KIND_ACT), T, K, outliers=outliers)
     q, s, bs = gpu_quant(x)
