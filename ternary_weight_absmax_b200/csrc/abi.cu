@@ -464,12 +464,8 @@ static bitnet_status gemm_impl(const bitnet_weight *w, const int8_t *q_dev, cons
     DeviceGlobals g;
     e = device_globals(&g);
     if (e != cudaSuccess) return cuda_fail(e, "device globals");
-    const bool uniform = (w->flags & BITNET_WEIGHT_UNIFORM_ROWS) != 0;
-    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    if (uniform && !acc_dev)  // weights decoded into tensor memory, 128-token tiles
-        e = launch_gemm_tc(w->data, w->rows, w->cols, q_dev, s_dev, T, y_dev, g, st);
-    else
-        e = launch_gemm(w->data, w->rows, w->cols, uniform, q_dev, s_dev, T, y_dev, acc_dev, g, st);
+    e = launch_gemm(w->data, w->rows, w->cols, (w->flags & BITNET_WEIGHT_UNIFORM_ROWS) != 0, q_dev, s_dev,
+                    T, y_dev, acc_dev, g, reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? BITNET_OK : cuda_fail(e, "gemm launch");
 }
 

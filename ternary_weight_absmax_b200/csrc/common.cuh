@@ -99,9 +99,6 @@ constexpr int kTcMinBatch = 4;  // from this batch on the dispatcher prefers it 
 bool gemv_tc_supported(int64_t rows, int64_t cols, int64_t B);
 cudaError_t launch_gemv_tc(const void *data, int64_t rows, int64_t cols, const int8_t *q, const float *s,
                            int64_t B, float *y, const DeviceGlobals &g, cudaStream_t st);
-// The same kernel over 128-token tiles (T >= 1 tokens, uniform rows): prefill.
-cudaError_t launch_gemm_tc(const void *data, int64_t rows, int64_t cols, const int8_t *q, const float *s,
-                           int64_t T, float *y, const DeviceGlobals &g, cudaStream_t st);
 // One linear of a sequence call (decode_seq.cu): repacked weight data with
 // uniform rows, fp32 x [cols], fp32 y [rows], and the index of the linear whose
 // y this x reads (-1: x is ready at launch).

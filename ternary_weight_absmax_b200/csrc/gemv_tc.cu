@@ -47,31 +47,33 @@ namespace bitnet {
 namespace {
 
 constexpr int kThreads = 192;     // 6 warps
-constexpr int kTmemCols = 256;    // accumulator at [0, NT), A buffers after it, 32 columns per stage
+constexpr int kTmemCols = 256;    // accumulator at [0, 64), A buffers at 64 + 32 * buffer
+constexpr int kAcol = 64;
+constexpr int kNA = 6;            // tensor-memory A buffers (one K block each)
 constexpr uint32_t kDrainLimit = 1u << 22;
 
-// NT tokens per CTA: 16, 32, 64 (GEMV; K may be split over a cluster) or 128
-// (prefill tiles; no split).
+// NT tokens per CTA (16, 32 or 64).  The shared-memory ring is deeper than
+// the tensor-memory one: a stage lives from its copy until its MMAs finish,
+// most of it waiting on HBM, while an A buffer lives only from its decode to
+// its MMAs.  About 96 KB of stages per CTA, two CTAs per SM.
 template <int NT>
 struct TcCfg {
-    static constexpr int kStages = NT <= 64 ? 6 : 4;          // pipeline stages = tensor-memory A buffers
-    static constexpr int kAcol = NT <= 64 ? 64 : 128;         // first A-buffer column
-    static_assert(kAcol + 32 * kStages <= kTmemCols, "tensor-memory columns");
+    static constexpr int kStages = NT == 16 ? 16 : (NT == 32 ? 12 : 8);
     static constexpr int kQBytes = NT * 128;                  // activations of one block, 128-byte rows
     static constexpr int kCodeBytes = 8 * kTileBytes;         // eight 16-row code tiles of one block
     static constexpr int kStageBytes = kQBytes + kCodeBytes;  // multiple of 1024
-    static constexpr bool kSplit = NT <= 64;                  // K may be split over a cluster
-    static constexpr int kRedStride = NT + 1;                 // int32 per row of the cluster sum (+1: banks)
-    static constexpr int kOffRed = kStages * kStageBytes;
-    static constexpr int kOffSq = kOffRed + (kSplit ? 128 * kRedStride * 4 : 0);
+    static constexpr int kPartStride = NT + 1;                // int32 partial sums [128][NT + 1] (+1: banks)
+    static constexpr int kOffSq = kStages * kStageBytes;
     static constexpr int kOffInv = kOffSq + NT * 4;
     static constexpr int kOffBar = kOffInv + NT * 4;
     // At least 80 KB so that no more than two CTAs share an SM: two hold all
     // 512 tensor-memory columns, and a third would block in its allocation.
-    static constexpr size_t kUsed = 1024 + (size_t)kOffBar + 256;
+    static constexpr size_t kUsed = 1024 + (size_t)kOffBar + 512;
     static constexpr size_t kSmem = kUsed > 80 * 1024 ? kUsed : 80 * 1024;
     static_assert(kStageBytes % 1024 == 0, "stages keep 1024-byte alignment");
+    static_assert(128 * kPartStride * 4 <= kOffSq, "partial sums fit in the stages they reuse");
     static_assert(kSmem <= 110 * 1024, "two CTAs per SM");
+    static_assert(kAcol + 32 * kNA <= kTmemCols && NT <= kAcol, "tensor-memory columns");
 };
 
 struct TcArgs {
@@ -113,12 +115,17 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, uint32_
     return ok != 0;
 }
 
+__device__ __forceinline__ int ld_cluster_s32(uint32_t addr) {
+    int v;
+    asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+    return v;
+}
+
 template <int NT>
 __global__ void __launch_bounds__(kThreads, 2)
 gemv_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constant__ CUtensorMap map_q, const TcArgs a) {
     using C = TcCfg<NT>;
     constexpr int S = C::kStages;
-    constexpr int kAcol = C::kAcol;
     extern __shared__ unsigned char smem_raw[];
     const uint32_t raw = ptx::smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
@@ -126,19 +133,19 @@ gemv_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constant_
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = a.splits > 1 ? ptx::cluster_rank() : 0u;
     const int mt = (int)(blockIdx.x / (unsigned)a.splits);
-    const int b0 = (int)blockIdx.y * NT;            // first token of this CTA
-    const int bt = min(NT, a.B - b0);               // its tokens
+    const int bt = a.B;  // tokens (<= NT)
     const int j0 = (int)((int64_t)rank * a.nb / a.splits);
     const int nj = (int)((int64_t)(rank + 1) * a.nb / a.splits) - j0;
     const uint32_t bars = base + C::kOffBar;
     auto full = [&](int s) { return bars + 8u * s; };
     auto empty = [&](int s) { return bars + 8u * (S + s); };
-    auto decb = [&](int s) { return bars + 8u * (2 * S + s); };
-    const uint32_t accf = bars + 8u * (3 * S);
-    const uint32_t drain = bars + 8u * (3 * S + 1);
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(gbase + C::kOffBar + 8 * (3 * S + 2));
+    auto decb = [&](int b) { return bars + 8u * (2 * S + b); };
+    auto afree = [&](int b) { return bars + 8u * (2 * S + kNA + b); };
+    const uint32_t accf = bars + 8u * (2 * S + 2 * kNA);
+    const uint32_t drain = accf + 8u;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(gbase + C::kOffBar + 8 * (2 * S + 2 * kNA + 2));
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-    int *red = reinterpret_cast<int *>(gbase + C::kOffRed);
+    int *part = reinterpret_cast<int *>(gbase);  // [128][kPartStride], after the main loop
     int *sq = reinterpret_cast<int *>(gbase + C::kOffSq);
     float *inv = reinterpret_cast<float *>(gbase + C::kOffInv);
     const uint32_t limit = *a.wait_limit;
@@ -147,7 +154,10 @@ gemv_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constant_
         for (int s = 0; s < S; s++) {
             ptx::mbar_init(full(s), 1);
             ptx::mbar_init(empty(s), 1);
-            ptx::mbar_init(decb(s), 4);
+        }
+        for (int b = 0; b < kNA; b++) {
+            ptx::mbar_init(decb(b), 4);
+            ptx::mbar_init(afree(b), 1);
         }
         ptx::mbar_init(accf, 1);
         ptx::mbar_init(drain, 1);
@@ -160,15 +170,11 @@ gemv_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constant_
         ptx::tmem_alloc(ptx::smem_u32(tmem_slot), kTmemCols);
         ptx::tmem_relinquish();
     }
-    if (C::kSplit)
-        for (int i = threadIdx.x; i < 128 * C::kRedStride; i += kThreads) red[i] = 0;
     for (int i = threadIdx.x; i < NT; i += kThreads) sq[i] = 0;
     ptx::tc_fence_before();
     __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    // The first CTA's sum buffer is zero before any CTA of the cluster adds to it.
-    if (C::kSplit && a.splits > 1) ptx::cluster_sync();
 
     auto give_up = [&]() {
         *abort_flag = 1;
@@ -189,19 +195,17 @@ gemv_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constant_
         // ------------------------------------------------ TMA producer
         if (lane == 0) {
             int issued = 0;
-            bool ok = true;
             for (int it = 0; it < nj; it++) {
                 const int s = it % S;
                 if (it >= S) {
                     if (!ptx::mbar_wait(empty(s), ((it / S) - 1) & 1, limit, abort_flag)) {
                         give_up();
-                        ok = false;
                         break;
                     }
                     ptx::mbar_arrive_expect_tx(full(s), C::kCodeBytes + C::kQBytes);
                     ptx::tma_load_3d(base + s * C::kStageBytes + C::kQBytes, &map_c, full(s), 0, j0 + it, mt * 8);
                 }
-                ptx::tma_load_2d(base + s * C::kStageBytes, &map_q, full(s), 128 * (j0 + it), b0);
+                ptx::tma_load_2d(base + s * C::kStageBytes, &map_q, full(s), 128 * (j0 + it), 0);
                 issued = it + 1;
             }
             // Copies in flight (the last S stages issued) land before the CTA
@@ -209,7 +213,6 @@ gemv_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constant_
             // issued before it has both of its copies.
             for (int it = issued > S ? issued - S : 0; it < issued; it++)
                 ptx::mbar_wait(full(it % S), (it / S) & 1, kDrainLimit, nullptr);
-            (void)ok;
         }
         __syncwarp();
     } else if (warp == 1) {
@@ -217,18 +220,19 @@ gemv_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constant_
         if (lane == 0) {
             constexpr uint32_t idesc = ptx::idesc_i8(128, NT, false);
             for (int it = 0; it < nj; it++) {
-                const int s = it % S;
-                if (!ptx::mbar_wait(decb(s), (it / S) & 1, limit, abort_flag)) {
+                const int s = it % S, ab = it % kNA;
+                if (!ptx::mbar_wait(decb(ab), (it / kNA) & 1, limit, abort_flag)) {
                     give_up();
                     break;
                 }
                 ptx::tc_fence_after();
                 const uint64_t bdesc = ptx::desc_k_sw128(base + s * C::kStageBytes);
-                const uint32_t acol = tmem + (uint32_t)(kAcol + 32 * s);
+                const uint32_t acol = tmem + (uint32_t)(kAcol + 32 * ab);
 #pragma unroll
                 for (int gg = 0; gg < 4; gg++)
                     ptx::mma_i8_ta(tmem, acol + 8u * gg, bdesc + 2u * gg, idesc, (it > 0 || gg > 0) ? 1u : 0u);
                 ptx::mma_commit(empty(s));
+                ptx::mma_commit(afree(ab));
             }
             ptx::mma_commit(accf);
             ptx::mma_commit(drain);
@@ -239,32 +243,35 @@ gemv_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constant_
         // ------------------------------------------------ decoders, then epilogue
         const int quarter = warp & 3;  // tensor-memory lanes 32 * quarter ..
         const uint32_t tlane = (uint32_t)(quarter * 32) << 16;
-        const int d = threadIdx.x - 64;                 // 0..127
-        constexpr int kPer = 128 / NT;                  // threads per token for sum(q)
-        const int tok = d / kPer, part = d % kPer;
-        if (d < bt) inv[d] = __frcp_rn(a.s[b0 + d]);
+        const int d = threadIdx.x - 64;  // 0..127
+        constexpr int kPer = 128 / NT;   // threads per token for sum(q)
+        const int tok = d / kPer, part_i = d % kPer;
+        if (d < bt) inv[d] = __frcp_rn(a.s[d]);
         const int row = quarter * 32 + lane;
         const int64_t o = (int64_t)mt * 128 + row;
-        const float rs = o < a.rows ? __ldg(a.rowscale + o) : 0.0f;
+        const float rs = a.splits == 1 && o < a.rows ? __ldg(a.rowscale + o) : 0.0f;
         int sqa = 0;
         bool ok = true;
-        for (int it = 0; it < nj && ok; it++) {
-            const int s = it % S;
-            if (!warp_wait<false>(full(s), (it / S) & 1, limit, abort_flag)) {
+        for (int it = 0; it < nj; it++) {
+            const int s = it % S, ab = it % kNA;
+            if (!warp_wait<false>(full(s), (it / S) & 1, limit, abort_flag) ||
+                (it >= kNA && !warp_wait<false>(afree(ab), ((it / kNA) - 1) & 1, limit, abort_flag))) {
                 if (lane == 0) give_up();
                 ok = false;
                 break;
             }
+            ptx::tc_fence_after();
             const unsigned char *st = gbase + s * C::kStageBytes;
             const uint4 *cs = reinterpret_cast<const uint4 *>(st + C::kQBytes);
+            const uint32_t acol = tmem + tlane + (uint32_t)(kAcol + 32 * ab);
             uint32_t v[16];
             decode_tile(cs[(2 * quarter) * 32 + lane], v);
-            ptx::tmem_st_16x128b_x8(tmem + tlane + (uint32_t)(kAcol + 32 * s), v);
+            ptx::tmem_st_16x128b_x8(acol, v);
             decode_tile(cs[(2 * quarter + 1) * 32 + lane], v);
-            ptx::tmem_st_16x128b_x8(tmem + tlane + (16u << 16) + (uint32_t)(kAcol + 32 * s), v);
+            ptx::tmem_st_16x128b_x8(acol + (16u << 16), v);
             // sum(q) of token `tok`: its 128-byte row of the stage (the swizzle
             // permutes 16-byte chunks within the row), NT bytes per thread.
-            const uint4 *qr = reinterpret_cast<const uint4 *>(st + tok * 128 + part * NT);
+            const uint4 *qr = reinterpret_cast<const uint4 *>(st + tok * 128 + part_i * NT);
 #pragma unroll
             for (int c = 0; c < NT / 16; c++) {
                 const uint4 qv = qr[c];
@@ -276,52 +283,60 @@ gemv_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constant_
             ptx::tmem_wait_st();
             ptx::tc_fence_before();
             __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(decb(s));
+            if (lane == 0) ptx::mbar_arrive(decb(ab));
         }
         atomicAdd(sq + tok, sqa);
         asm volatile("bar.sync 1, 128;" ::: "memory");  // sum(q) and 1/s complete (decoder warps only)
-        // The accumulator, 16 token columns at a time (thread = row): sum t*q =
-        // sum c*q - sum q; then y (no split) or an add into the first CTA.
-        if (ok && warp_wait<true>(accf, 0, limit, abort_flag)) {
-            ptx::tc_fence_after();
-            const uint32_t dst = C::kSplit && a.splits > 1
-                                     ? ptx::map_to_rank(ptx::smem_u32(red + row * C::kRedStride), 0)
-                                     : 0u;
+        // The accumulator, 16 token columns at a time (thread = row):
+        // sum t*q = sum c*q - sum q; then y (no split) or this CTA's partial
+        // sums (the stages are free once every MMA has completed).
+        const bool have = ok && warp_wait<true>(accf, 0, limit, abort_flag);
+        if (ok && !have && lane == 0) give_up();
+        if (have) ptx::tc_fence_after();
 #pragma unroll 1
-            for (int c0 = 0; c0 < NT && c0 < bt; c0 += 16) {
-                uint32_t v[16];
+        for (int c0 = 0; c0 < NT && c0 < bt; c0 += 16) {
+            uint32_t v[16];
+            if (have) {
                 ptx::tmem_ld_32x32b_x16(tmem + tlane + (uint32_t)c0, v);
                 ptx::tmem_wait_ld();
+            } else {
 #pragma unroll
-                for (int i = 0; i < 16; i++) {
-                    const int b = c0 + i;
-                    if (b >= bt) break;
-                    const int val = (int)v[i] - sq[b];
-                    if (!C::kSplit || a.splits == 1) {
-                        if (o < a.rows)
-                            a.y[(int64_t)(b0 + b) * a.rows + o] = __fmul_rn(__fmul_rn(rs, (float)val), inv[b]);
-                    } else {
-                        ptx::red_add_cluster(dst + 4u * b, val);
-                    }
+                for (int i = 0; i < 16; i++) v[i] = 0u;
+            }
+#pragma unroll
+            for (int i = 0; i < 16; i++) {
+                const int b = c0 + i;
+                if (b >= bt) break;
+                const int val = (int)v[i] - sq[b];
+                if (a.splits == 1) {
+                    if (o < a.rows) a.y[(int64_t)b * a.rows + o] = __fmul_rn(__fmul_rn(rs, (float)val), inv[b]);
+                } else {
+                    part[row * C::kPartStride + b] = val;
                 }
             }
-        } else if (ok && lane == 0) {
-            give_up();
         }
     }
 
-    if (C::kSplit && a.splits > 1) {
-        ptx::cluster_sync();  // every CTA's partial sums have landed in the first CTA
-        if (rank == 0 && warp >= 2) {
-            const int row = (warp & 3) * 32 + lane;
+    if (a.splits > 1) {
+        // Every CTA's partial sums are in its shared memory; CTA r sums rows
+        // [r R, r R + R) over the cluster (R = 128 / splits) and writes y.
+        ptx::cluster_sync();
+        if (warp >= 2) {
+            const int d = threadIdx.x - 64;
+            const int R = 128 / a.splits;
+            const int row = (int)rank * R + d % R;
             const int64_t o = (int64_t)mt * 128 + row;
             if (o < a.rows) {
                 const float rs = __ldg(a.rowscale + o);
-                for (int b = 0; b < bt; b++)
-                    a.y[(int64_t)(b0 + b) * a.rows + o] =
-                        __fmul_rn(__fmul_rn(rs, (float)red[row * C::kRedStride + b]), inv[b]);
+                const uint32_t loc = ptx::smem_u32(part + row * C::kPartStride);
+                for (int b = d / R; b < bt; b += 128 / R) {
+                    int v = 0;
+                    for (int k = 0; k < a.splits; k++) v += ld_cluster_s32(ptx::map_to_rank(loc + 4u * b, (uint32_t)k));
+                    a.y[(int64_t)b * a.rows + o] = __fmul_rn(__fmul_rn(rs, (float)v), inv[b]);
+                }
             }
         }
+        ptx::cluster_sync();  // no CTA leaves while another reads its partial sums
     }
     ptx::tc_fence_before();
     __syncthreads();
@@ -384,7 +399,7 @@ cudaError_t run_tc(const void *data, const Layout &L, const int8_t *q, TcArgs a,
     }
     const int64_t mtiles = (L.rows + 127) / 128;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(mtiles * a.splits), (unsigned)((a.B + NT - 1) / NT));
+    cfg.gridDim = dim3((unsigned)(mtiles * a.splits));
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = C::kSmem;
     cfg.stream = st;
@@ -407,23 +422,6 @@ bool gemv_tc_supported(int64_t rows, int64_t cols, int64_t B) {
     return B >= 1 && B <= 64 && cols >= kQK && cols <= (int64_t(1) << 17);
 }
 
-cudaError_t launch_gemm_tc(const void *data, int64_t rows, int64_t cols, const int8_t *q, const float *s,
-                           int64_t T, float *y, const DeviceGlobals &g, cudaStream_t st) {
-    const Layout L = layout_of(rows, cols);
-    const unsigned char *base = static_cast<const unsigned char *>(data);
-    TcArgs a;
-    a.rowscale = reinterpret_cast<const float *>(base + L.off_rowscale);
-    a.s = s;
-    a.y = y;
-    a.err = g.err;
-    a.wait_limit = g.wait_limit;
-    a.rows = rows;
-    a.B = (int)T;
-    a.nb = (int)L.nb;
-    a.splits = 1;
-    return run_tc<128>(data, L, q, a, st);
-}
-
 cudaError_t launch_gemv_tc(const void *data, int64_t rows, int64_t cols, const int8_t *q, const float *s,
                            int64_t B, float *y, const DeviceGlobals &g, cudaStream_t st) {
     const Layout L = layout_of(rows, cols);
@@ -437,10 +435,11 @@ cudaError_t launch_gemv_tc(const void *data, int64_t rows, int64_t cols, const i
     a.rows = rows;
     a.B = (int)B;
     a.nb = (int)L.nb;
-    // K split over a cluster so that the grid fills two CTAs per SM in one wave.
+    // K split over a cluster so that the grid fills two CTAs per SM in one
+    // wave, keeping at least four K blocks per CTA.
     const int64_t mtiles = (rows + 127) / 128;
     int splits = 1;
-    while (splits < 8 && splits * 2 <= a.nb && mtiles * splits * 2 <= 2 * (int64_t)num_sms()) splits *= 2;
+    while (splits < 8 && a.nb / (splits * 2) >= 4 && mtiles * splits * 2 <= 2 * (int64_t)num_sms()) splits *= 2;
     a.splits = splits;
     if (B <= 16) return run_tc<16>(data, L, q, a, st);
     if (B <= 32) return run_tc<32>(data, L, q, a, st);
