@@ -34,7 +34,8 @@
 //      tiles split between warps are summed in shared memory;
 //   C  the split tiles' rows are written; if a later linear reads this
 //      linear's y, the CTA adds its tile count to the linear's counter in the
-//      caller's workspace (release), which the consumers poll (acquire).
+//      caller's workspace, and the CTA that completes the count raises the
+//      linear's ready word (release), which the consumers poll (acquire).
 // Linears without a producer thus overlap freely (a CTA holds a contiguous
 // slice of the wave, usually one to three linears); a chain of dependent
 // linears pays one grid-wide hand-off per linear but never waits for weights.
@@ -66,7 +67,7 @@ constexpr int kRingBytes = kWarps * kSlots * kChunk * kTile;  // 192 KB
 constexpr int kOffQ = kOffRing + kRingBytes;                  // q, K bytes (permuted words)
 constexpr int kOffAcc = kOffQ + kSeqMaxK;                     // [kSmallTiles * 16] int32
 constexpr int kOffSeg = kOffAcc + kSmallTiles * kTileRows * 4;
-constexpr int kOffRed = kOffSeg + 2 * kSeqMaxLinears * 4;     // absmax bits, sum(q), abort flag
+constexpr int kOffRed = kOffSeg + 3 * kSeqMaxLinears * 4 + 64;  // absmax bits, sum(q), abort flag
 constexpr int kOffBar = kOffRed + 64;
 constexpr int kSmem = kOffBar + kWarps * kSlots * 8;
 static_assert(kSmem <= 227 * 1024, "shared memory");
@@ -85,6 +86,7 @@ struct SeqLin {
 
 struct SeqArgs {
     unsigned *done;        // [n] tiles finished per linear (workspace), or null
+    unsigned *ready;       // [n] set to 1 by the CTA that completes a linear (workspace), or null
     unsigned *exit_count;  // CTAs finished (workspace), or null
     unsigned *abort;       // set by a CTA that gave up, so the others stop waiting (workspace), or null
     unsigned *err;
@@ -110,6 +112,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_seq_kernel(const __grid_co
     const int c = blockIdx.x, G = gridDim.x;
     int *seg_lo = reinterpret_cast<int *>(smem + kOffSeg);
     int *seg_cnt = seg_lo + kSeqMaxLinears;
+    int *seg_list = seg_cnt + kSeqMaxLinears;  // linears with tiles in this CTA, in list order
+    int *seg_wcnt = seg_list + kSeqMaxLinears; // [8] + count
     uint32_t *qw = reinterpret_cast<uint32_t *>(smem + kOffQ);
     int *acc = reinterpret_cast<int *>(smem + kOffAcc);
     unsigned *amax_w = reinterpret_cast<unsigned *>(smem + kOffRed);
@@ -142,6 +146,20 @@ __global__ void __launch_bounds__(kThreads, 1) decode_seq_kernel(const __grid_co
         ptx::fence_mbar_init();
     }
     __syncthreads();
+    // Compact list of this CTA's segments (warp ballots; n <= 256 = 8 warps).
+    const int cL = warp * 32 + lane;
+    const bool has = warp < kSeqMaxLinears / 32 && cL < n && seg_cnt[cL] > 0;
+    const unsigned hmask = __ballot_sync(0xffffffffu, has);
+    if (warp < kSeqMaxLinears / 32 && lane == 0) seg_wcnt[warp] = __popc(hmask);
+    __syncthreads();
+    if (warp < kSeqMaxLinears / 32) {
+        int before = 0;
+        for (int w = 0; w < warp; w++) before += seg_wcnt[w];
+        if (has) seg_list[before + __popc(hmask & ((1u << lane) - 1u))] = cL;
+        if (warp == kSeqMaxLinears / 32 - 1 && lane == 0) seg_wcnt[kSeqMaxLinears / 32] = before + __popc(hmask);
+    }
+    __syncthreads();
+    const int nseg = seg_wcnt[kSeqMaxLinears / 32];
 
     // This warp's items of segment L: [i0, i1) of the segment's cnt * nb.
     auto run_of = [&](int L, int &i0, int &i1) {
@@ -152,14 +170,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_seq_kernel(const __grid_co
 
     // ---- issue cursor (lane 0): the next chunk of this warp's item stream.
     const uint64_t pol = ptx::policy_evict_first();
-    int iL = -1, ii = 0, iend = 0;  // linear, next item, end of its run
-    uint32_t iq = 0;                // chunks issued
+    int ik = -1, iL = -1, ii = 0, iend = 0;  // segment, its linear, next item, end of its run
+    uint32_t iq = 0;                         // chunks issued
     auto next_run = [&]() {
-        while (++iL < n) {
-            if (seg_cnt[iL] == 0) continue;
+        while (++ik < nseg) {
+            iL = seg_list[ik];
             run_of(iL, ii, iend);
             if (iend > ii) return;
         }
+        iL = n;
     };
     auto issue = [&]() {
         if (iL >= n) return;
@@ -183,9 +202,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_seq_kernel(const __grid_co
     bool ok = true;
     const uint4 *qrow = reinterpret_cast<const uint4 *>(qw + t * 8);  // block 0, this lane's part
 
-    for (int L = 0; L < n; L++) {
+    for (int k = 0; k < nseg; k++) {
+        const int L = seg_list[k];
         const int cnt = seg_cnt[L];
-        if (cnt == 0) continue;
         const SeqLin &l = a.lin[L];
         const int nb = l.nb, rlo = seg_lo[L];
         const int64_t items = (int64_t)cnt * nb;
@@ -213,11 +232,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_seq_kernel(const __grid_co
             // Each poll is an L2 round trip: a sixteenth of the copy-wait
             // iteration cap and the wall-clock cap bound the wait; another
             // CTA's abort ends it at once.
-            const unsigned need = (unsigned)a.lin[l.dep].ntr;
             const uint32_t dlim = limit >> 4 ? limit >> 4 : 1u;
             uint32_t it = 0;
             ptx::WaitClock clk;
-            while (ld_acquire_gpu(a.done + l.dep) < need) {
+            while (ld_acquire_gpu(a.ready + l.dep) == 0u) {
                 if (++it >= dlim || clk.expired(it) || *reinterpret_cast<volatile unsigned *>(a.abort)) {
                     *bad_w = 1;
                     atomicOr(a.err, kErrTimeout);
@@ -241,11 +259,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_seq_kernel(const __grid_co
             }
         }
         // The next segment's x, if it is ready at launch, into L2 meanwhile.
-        for (int L2 = L + 1; L2 < n; L2++) {
-            if (seg_cnt[L2] == 0) continue;
-            if (a.lin[L2].dep < 0)
-                for (int i = tid; i < a.lin[L2].nb * 4; i += kThreads) prefetch_l2(a.lin[L2].x + i * 32);
-            break;
+        if (k + 1 < nseg && a.lin[seg_list[k + 1]].dep < 0) {
+            const SeqLin &l2 = a.lin[seg_list[k + 1]];
+            for (int i = tid; i < l2.nb * 4; i += kThreads) prefetch_l2(l2.x + i * 32);
         }
         // m >= 0 and not NaN (fmaxf drops NaN): its bit pattern orders like its value.
         const unsigned mu = __reduce_max_sync(0xffffffffu, __float_as_uint(m));
@@ -370,7 +386,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_seq_kernel(const __grid_co
             __syncthreads();
             if (tid == 0 && !*bad_w) {
                 __threadfence();
-                atomicAdd(a.done + L, (unsigned)cnt);
+                // The CTA whose tiles complete the linear publishes it: the
+                // consumers poll a word written once, not the counter the
+                // producers are adding to.
+                const unsigned prev = atomicAdd(a.done + L, (unsigned)cnt);
+                if (prev + (unsigned)cnt == (unsigned)l.ntr) {
+                    __threadfence();
+                    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(a.ready + L), "r"(1u) : "memory");
+                }
             }
         }
     }
@@ -387,7 +410,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_seq_kernel(const __grid_co
         const unsigned prev = atomicAdd(a.exit_count, 1u);
         if (prev == (unsigned)G - 1) {  // every other CTA is past its last wait
             __threadfence();
-            for (int L = 0; L < n; L++) a.done[L] = 0u;
+            for (int L = 0; L < n; L++) a.done[L] = a.ready[L] = 0u;
             *a.exit_count = 0u;
             *a.abort = 0u;
             __threadfence();
@@ -397,7 +420,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_seq_kernel(const __grid_co
 
 }  // namespace
 
-size_t seq_workspace_bytes(int n) { return align_up((size_t)(n + 2) * sizeof(unsigned), 256); }
+size_t seq_workspace_bytes(int n) { return align_up((size_t)(2 * n + 2) * sizeof(unsigned), 256); }
 
 cudaError_t launch_decode_seq(const SeqLinear *list, int n, void *workspace, const DeviceGlobals &g,
                               cudaStream_t st) {
@@ -447,8 +470,9 @@ cudaError_t launch_decode_seq(const SeqLinear *list, int n, void *workspace, con
         if (list[i].dep >= 0) a.lin[list[i].dep].signal = 1;
     unsigned *ws = static_cast<unsigned *>(workspace);
     a.done = any_dep ? ws : nullptr;
-    a.exit_count = any_dep ? ws + n : nullptr;
-    a.abort = any_dep ? ws + n + 1 : nullptr;
+    a.ready = any_dep ? ws + n : nullptr;
+    a.exit_count = any_dep ? ws + 2 * n : nullptr;
+    a.abort = any_dep ? ws + 2 * n + 1 : nullptr;
 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)num_sms());
