@@ -180,11 +180,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_seq_kernel(const __grid_co
         }
         iL = n;
     };
+    uint32_t islot = 0;  // slot of the next chunk issued (iq mod kSlots)
     auto issue = [&]() {
         if (iL >= n) return;
         const SeqLin &l = a.lin[iL];
         const int nt = min(kChunk, iend - ii);
-        const uint32_t slot = iq % kSlots;
+        const uint32_t slot = islot;
+        islot = islot + 1 == kSlots ? 0u : islot + 1;
         const uint32_t bar = bar0 + 8u * slot;
         ptx::mbar_arrive_expect_tx(bar, (uint32_t)(nt * kTile));
         ptx::bulk_g2s(ptx::smem_u32(ring + slot * (kChunk * kTile)),
@@ -198,7 +200,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_seq_kernel(const __grid_co
         for (int k = 0; k < kSlots; k++) issue();
     }
 
-    uint32_t cq = 0;  // chunks consumed (every lane keeps the same count)
+    uint32_t cq = 0;                      // chunks consumed (every lane keeps the same count)
+    uint32_t cslot = 0, cphase = 0;       // its slot and the parity of that slot's phase
     bool ok = true;
     const uint4 *qrow = reinterpret_cast<const uint4 *>(qw + t * 8);  // block 0, this lane's part
 
@@ -325,12 +328,26 @@ __global__ void __launch_bounds__(kThreads, 1) decode_seq_kernel(const __grid_co
                         ? __ldg(l.rowscale + (int64_t)(rlo + r + kRsDepth) * kTileRows + (lane & 15))
                         : 0.0f;
             };
+            // The products of one item: tile word w (this lane's 16 bytes),
+            // activation words at q (qa0 qb0 qa1 qb1 | qa2 qb2 qa3 qb3).
+            auto item = [&](const uint4 w, const uint4 *q) {
+                const uint4 q0 = q[0], q1 = q[1];
+                const int qa[4] = {(int)q0.x, (int)q0.z, (int)q1.x, (int)q1.z};
+                const int qb[4] = {(int)q0.y, (int)q0.w, (int)q1.y, (int)q1.w};
+#pragma unroll
+                for (int gg = 0; gg < 4; gg++) {
+                    const uint32_t mk = 0xC0C0C0C0u >> (2 * gg);
+                    aA[gg] = dp4a_us(w.x & mk, qa[gg], aA[gg]);
+                    aA[gg] = dp4a_us(w.z & mk, qb[gg], aA[gg]);
+                    aB[gg] = dp4a_us(w.y & mk, qa[gg], aB[gg]);
+                    aB[gg] = dp4a_us(w.w & mk, qb[gg], aB[gg]);
+                }
+            };
             int i = i0;
             while (i < i1) {
-                const uint32_t slot = cq % kSlots;
+                const uint32_t slot = cslot;
                 int got = 1;
-                if (lane == 0)
-                    got = ptx::mbar_wait(bar0 + 8u * slot, (cq / kSlots) & 1u, limit, bad_w) ? 1 : 0;
+                if (lane == 0) got = ptx::mbar_wait(bar0 + 8u * slot, cphase, limit, bad_w) ? 1 : 0;
                 if (!__shfl_sync(0xffffffffu, got, 0)) {
                     if (lane == 0 && !*bad_w) {
                         *bad_w = 1;
@@ -342,29 +359,30 @@ __global__ void __launch_bounds__(kThreads, 1) decode_seq_kernel(const __grid_co
                 }
                 const int nt = min(kChunk, i1 - i);
                 const uint4 *wv = reinterpret_cast<const uint4 *>(ring + slot * (kChunk * kTile)) + lane;
-                for (int e = 0; e < nt; e++) {
-                    const uint4 w = wv[e * 32];
-                    const uint4 q0 = qp[0], q1 = qp[1];
-                    const int qa[4] = {(int)q0.x, (int)q0.z, (int)q1.x, (int)q1.z};
-                    const int qb[4] = {(int)q0.y, (int)q0.w, (int)q1.y, (int)q1.w};
+                if (nt == kChunk && j + kChunk < nb) {
+                    // A whole chunk inside the current row tile: no tile change.
 #pragma unroll
-                    for (int gg = 0; gg < 4; gg++) {
-                        const uint32_t mk = 0xC0C0C0C0u >> (2 * gg);
-                        aA[gg] = dp4a_us(w.x & mk, qa[gg], aA[gg]);
-                        aA[gg] = dp4a_us(w.z & mk, qb[gg], aA[gg]);
-                        aB[gg] = dp4a_us(w.y & mk, qa[gg], aB[gg]);
-                        aB[gg] = dp4a_us(w.w & mk, qb[gg], aB[gg]);
-                    }
-                    qp += 8;
-                    if (++j == nb) {
-                        flush();
-                        r++;
-                        j = 0;
-                        qp = qrow;
+                    for (int e = 0; e < kChunk; e++) item(wv[e * 32], qp + e * 8);
+                    qp += kChunk * 8;
+                    j += kChunk;
+                } else {
+                    for (int e = 0; e < nt; e++) {
+                        item(wv[e * 32], qp);
+                        qp += 8;
+                        if (++j == nb) {
+                            flush();
+                            r++;
+                            j = 0;
+                            qp = qrow;
+                        }
                     }
                 }
                 i += nt;
                 cq++;
+                if (++cslot == kSlots) {
+                    cslot = 0;
+                    cphase ^= 1u;
+                }
                 __syncwarp();  // every lane has read the slot
                 if (lane == 0) {
                     ptx::fence_proxy_async_smem();

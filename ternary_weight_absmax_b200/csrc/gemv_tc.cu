@@ -46,7 +46,9 @@
 namespace bitnet {
 namespace {
 
-constexpr int kThreads = 192;     // 6 warps
+constexpr int kDecSets = 2;       // decoder warp sets (4 warps each), taking K blocks in turn
+constexpr int kDecBatch = 2;      // K blocks a set decodes per wait for its tensor-memory stores
+constexpr int kThreads = 64 + 128 * kDecSets;  // producer, MMA, decoders (the first set also the epilogue)
 constexpr int kTmemCols = 256;    // accumulator at [0, 64), A buffers at 64 + 32 * buffer
 constexpr int kAcol = 64;
 constexpr int kNA = 6;            // tensor-memory A buffers (one K block each)
@@ -241,77 +243,90 @@ gemv_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constant_
         __syncwarp();
     } else {
         // ------------------------------------------------ decoders, then epilogue
+        // Set `set` decodes K blocks it = (kDecSets * m + set) * kDecBatch + u;
+        // within a set, kDecBatch blocks share one wait for the tensor-memory
+        // stores before they are handed to the MMA warp.
+        const int set = (warp - 2) >> 2;
         const int quarter = warp & 3;  // tensor-memory lanes 32 * quarter ..
         const uint32_t tlane = (uint32_t)(quarter * 32) << 16;
-        const int d = threadIdx.x - 64;  // 0..127
+        const int d = (threadIdx.x - 64) & 127;  // 0..127 within the set
         constexpr int kPer = 128 / NT;   // threads per token for sum(q)
         const int tok = d / kPer, part_i = d % kPer;
-        if (d < bt) inv[d] = __frcp_rn(a.s[d]);
+        if (set == 0 && d < bt) inv[d] = __frcp_rn(a.s[d]);
         const int row = quarter * 32 + lane;
         const int64_t o = (int64_t)mt * 128 + row;
         const float rs = a.splits == 1 && o < a.rows ? __ldg(a.rowscale + o) : 0.0f;
         int sqa = 0;
         bool ok = true;
-        for (int it = 0; it < nj; it++) {
-            const int s = it % S, ab = it % kNA;
-            if (!warp_wait<false>(full(s), (it / S) & 1, limit, abort_flag) ||
-                (it >= kNA && !warp_wait<false>(afree(ab), ((it / kNA) - 1) & 1, limit, abort_flag))) {
-                if (lane == 0) give_up();
-                ok = false;
-                break;
-            }
-            ptx::tc_fence_after();
-            const unsigned char *st = gbase + s * C::kStageBytes;
-            const uint4 *cs = reinterpret_cast<const uint4 *>(st + C::kQBytes);
-            const uint32_t acol = tmem + tlane + (uint32_t)(kAcol + 32 * ab);
-            uint32_t v[16];
-            decode_tile(cs[(2 * quarter) * 32 + lane], v);
-            ptx::tmem_st_16x128b_x8(acol, v);
-            decode_tile(cs[(2 * quarter + 1) * 32 + lane], v);
-            ptx::tmem_st_16x128b_x8(acol + (16u << 16), v);
-            // sum(q) of token `tok`: its 128-byte row of the stage (the swizzle
-            // permutes 16-byte chunks within the row), NT bytes per thread.
-            const uint4 *qr = reinterpret_cast<const uint4 *>(st + tok * 128 + part_i * NT);
+        for (int it0 = set * kDecBatch; it0 < nj && ok; it0 += kDecSets * kDecBatch) {
+            const int nd = min(kDecBatch, nj - it0);
+            for (int u = 0; u < nd; u++) {
+                const int it = it0 + u;
+                const int s = it % S, ab = it % kNA;
+                if (!warp_wait<false>(full(s), (it / S) & 1, limit, abort_flag) ||
+                    (it >= kNA && !warp_wait<false>(afree(ab), ((it / kNA) - 1) & 1, limit, abort_flag))) {
+                    if (lane == 0) give_up();
+                    ok = false;
+                    break;
+                }
+                ptx::tc_fence_after();
+                const unsigned char *st = gbase + s * C::kStageBytes;
+                const uint4 *cs = reinterpret_cast<const uint4 *>(st + C::kQBytes);
+                const uint32_t acol = tmem + tlane + (uint32_t)(kAcol + 32 * ab);
+                uint32_t v[16];
+                decode_tile(cs[(2 * quarter) * 32 + lane], v);
+                ptx::tmem_st_16x128b_x8(acol, v);
+                decode_tile(cs[(2 * quarter + 1) * 32 + lane], v);
+                ptx::tmem_st_16x128b_x8(acol + (16u << 16), v);
+                // sum(q) of token `tok`: its 128-byte row of the stage (the
+                // swizzle permutes 16-byte chunks within the row), NT bytes per
+                // thread.
+                const uint4 *qr = reinterpret_cast<const uint4 *>(st + tok * 128 + part_i * NT);
 #pragma unroll
-            for (int c = 0; c < NT / 16; c++) {
-                const uint4 qv = qr[c];
-                sqa = dp4a_ss((int)qv.x, 0x01010101, sqa);
-                sqa = dp4a_ss((int)qv.y, 0x01010101, sqa);
-                sqa = dp4a_ss((int)qv.z, 0x01010101, sqa);
-                sqa = dp4a_ss((int)qv.w, 0x01010101, sqa);
+                for (int c = 0; c < NT / 16; c++) {
+                    const uint4 qv = qr[c];
+                    sqa = dp4a_ss((int)qv.x, 0x01010101, sqa);
+                    sqa = dp4a_ss((int)qv.y, 0x01010101, sqa);
+                    sqa = dp4a_ss((int)qv.z, 0x01010101, sqa);
+                    sqa = dp4a_ss((int)qv.w, 0x01010101, sqa);
+                }
             }
+            if (!ok) break;
             ptx::tmem_wait_st();
             ptx::tc_fence_before();
             __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(decb(ab));
+            if (lane == 0)
+                for (int u = 0; u < nd; u++) ptx::mbar_arrive(decb((it0 + u) % kNA));
         }
         atomicAdd(sq + tok, sqa);
-        asm volatile("bar.sync 1, 128;" ::: "memory");  // sum(q) and 1/s complete (decoder warps only)
-        // The accumulator, 16 token columns at a time (thread = row):
-        // sum t*q = sum c*q - sum q; then y (no split) or this CTA's partial
-        // sums (the stages are free once every MMA has completed).
-        const bool have = ok && warp_wait<true>(accf, 0, limit, abort_flag);
-        if (ok && !have && lane == 0) give_up();
-        if (have) ptx::tc_fence_after();
+        asm volatile("bar.sync 1, %0;" ::"n"(128 * kDecSets) : "memory");  // sum(q), 1/s complete (decoders)
+        if (set == 0) {  // the first set writes the results
+            // The accumulator, 16 token columns at a time (thread = row):
+            // sum t*q = sum c*q - sum q; then y (no split) or this CTA's partial
+            // sums (the stages are free once every MMA has completed).
+            const bool have = ok && warp_wait<true>(accf, 0, limit, abort_flag);
+            if (ok && !have && lane == 0) give_up();
+            if (have) ptx::tc_fence_after();
 #pragma unroll 1
-        for (int c0 = 0; c0 < NT && c0 < bt; c0 += 16) {
-            uint32_t v[16];
-            if (have) {
-                ptx::tmem_ld_32x32b_x16(tmem + tlane + (uint32_t)c0, v);
-                ptx::tmem_wait_ld();
-            } else {
-#pragma unroll
-                for (int i = 0; i < 16; i++) v[i] = 0u;
-            }
-#pragma unroll
-            for (int i = 0; i < 16; i++) {
-                const int b = c0 + i;
-                if (b >= bt) break;
-                const int val = (int)v[i] - sq[b];
-                if (a.splits == 1) {
-                    if (o < a.rows) a.y[(int64_t)b * a.rows + o] = __fmul_rn(__fmul_rn(rs, (float)val), inv[b]);
+            for (int c0 = 0; c0 < NT && c0 < bt; c0 += 16) {
+                uint32_t v[16];
+                if (have) {
+                    ptx::tmem_ld_32x32b_x16(tmem + tlane + (uint32_t)c0, v);
+                    ptx::tmem_wait_ld();
                 } else {
-                    part[row * C::kPartStride + b] = val;
+#pragma unroll
+                    for (int i = 0; i < 16; i++) v[i] = 0u;
+                }
+#pragma unroll
+                for (int i = 0; i < 16; i++) {
+                    const int b = c0 + i;
+                    if (b >= bt) break;
+                    const int val = (int)v[i] - sq[b];
+                    if (a.splits == 1) {
+                        if (o < a.rows) a.y[(int64_t)b * a.rows + o] = __fmul_rn(__fmul_rn(rs, (float)val), inv[b]);
+                    } else {
+                        part[row * C::kPartStride + b] = val;
+                    }
                 }
             }
         }
@@ -321,7 +336,7 @@ gemv_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constant_
         // Every CTA's partial sums are in its shared memory; CTA r sums rows
         // [r R, r R + R) over the cluster (R = 128 / splits) and writes y.
         ptx::cluster_sync();
-        if (warp >= 2) {
+        if (warp >= 2 && warp < 6) {
             const int d = threadIdx.x - 64;
             const int R = 128 / a.splits;
             const int row = (int)rank * R + d % R;
