@@ -34,8 +34,8 @@
 //      tiles split between warps are summed in shared memory;
 //   C  the split tiles' rows are written; if a later linear reads this
 //      linear's y, the CTA adds its tile count to the linear's counter in the
-//      caller's workspace, and the CTA that completes the count raises the
-//      linear's ready word (release), which the consumers poll (acquire).
+//      caller's workspace (after a fence), which the consumers poll (acquire)
+//      until it reaches the linear's tile count.
 // Linears without a producer thus overlap freely (a CTA holds a contiguous
 // slice of the wave, usually one to three linears); a chain of dependent
 // linears pays one grid-wide hand-off per linear but never waits for weights.
@@ -86,7 +86,6 @@ struct SeqLin {
 
 struct SeqArgs {
     unsigned *done;        // [n] tiles finished per linear (workspace), or null
-    unsigned *ready;       // [n] set to 1 by the CTA that completes a linear (workspace), or null
     unsigned *exit_count;  // CTAs finished (workspace), or null
     unsigned *abort;       // set by a CTA that gave up, so the others stop waiting (workspace), or null
     unsigned *err;
@@ -238,7 +237,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_seq_kernel(const __grid_co
             const uint32_t dlim = limit >> 4 ? limit >> 4 : 1u;
             uint32_t it = 0;
             ptx::WaitClock clk;
-            while (ld_acquire_gpu(a.ready + l.dep) == 0u) {
+            const unsigned need = (unsigned)a.lin[l.dep].ntr;
+            while (ld_acquire_gpu(a.done + l.dep) < need) {
                 if (++it >= dlim || clk.expired(it) || *reinterpret_cast<volatile unsigned *>(a.abort)) {
                     *bad_w = 1;
                     atomicOr(a.err, kErrTimeout);
@@ -404,14 +404,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_seq_kernel(const __grid_co
             __syncthreads();
             if (tid == 0 && !*bad_w) {
                 __threadfence();
-                // The CTA whose tiles complete the linear publishes it: the
-                // consumers poll a word written once, not the counter the
-                // producers are adding to.
-                const unsigned prev = atomicAdd(a.done + L, (unsigned)cnt);
-                if (prev + (unsigned)cnt == (unsigned)l.ntr) {
-                    __threadfence();
-                    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(a.ready + L), "r"(1u) : "memory");
-                }
+                atomicAdd(a.done + L, (unsigned)cnt);
             }
         }
     }
@@ -428,7 +421,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_seq_kernel(const __grid_co
         const unsigned prev = atomicAdd(a.exit_count, 1u);
         if (prev == (unsigned)G - 1) {  // every other CTA is past its last wait
             __threadfence();
-            for (int L = 0; L < n; L++) a.done[L] = a.ready[L] = 0u;
+            for (int L = 0; L < n; L++) a.done[L] = 0u;
             *a.exit_count = 0u;
             *a.abort = 0u;
             __threadfence();
@@ -438,7 +431,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_seq_kernel(const __grid_co
 
 }  // namespace
 
-size_t seq_workspace_bytes(int n) { return align_up((size_t)(2 * n + 2) * sizeof(unsigned), 256); }
+size_t seq_workspace_bytes(int n) { return align_up((size_t)(n + 2) * sizeof(unsigned), 256); }
 
 cudaError_t launch_decode_seq(const SeqLinear *list, int n, void *workspace, const DeviceGlobals &g,
                               cudaStream_t st) {
@@ -488,9 +481,8 @@ cudaError_t launch_decode_seq(const SeqLinear *list, int n, void *workspace, con
         if (list[i].dep >= 0) a.lin[list[i].dep].signal = 1;
     unsigned *ws = static_cast<unsigned *>(workspace);
     a.done = any_dep ? ws : nullptr;
-    a.ready = any_dep ? ws + n : nullptr;
-    a.exit_count = any_dep ? ws + 2 * n : nullptr;
-    a.abort = any_dep ? ws + 2 * n + 1 : nullptr;
+    a.exit_count = any_dep ? ws + n : nullptr;
+    a.abort = any_dep ? ws + n + 1 : nullptr;
 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)num_sms());
