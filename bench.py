@@ -506,10 +506,14 @@ def run_llama8b(b, torch, dev, T, peaks):
                     res["b1_chain_seq"] = {"error": f"{type(e).__name__}: {e}"}
             else:
                 ents = linear_entries(weights, LAYERS_8B, SHAPES_8B, x_dev, xviews, ys)
-                g = T.capture(lambda: [b.bitnet_w2a8_linear(w, x, B, y) for (w, x, y, _) in ents])
-                res[f"b{B}_per_call"] = dict(hbm(nbytes, T.ms(g, 5), peak), launches=n_lin,
-                                             how="bitnet_w2a8_linear per linear (activation quantisation and "
-                                                 "the batched GEMV)")
+                maxk = max(k for _, _, k in SHAPES_8B)
+                qb = torch.empty(B * maxk, dtype=torch.int8, device=dev)
+                sb = torch.empty(B, dtype=torch.float32, device=dev)
+                g = T.capture(lambda: [b.bitnet_w2a8_linear(w, x, B, y, qb[:B * w.cols], sb)
+                                       for (w, x, y, _) in ents])
+                res[f"b{B}_per_call"] = dict(hbm(nbytes, T.ms(g, 5), peak), launches=2 * n_lin,
+                                             how="bitnet_w2a8_linear per linear with q_out / s_out: the "
+                                                 "quantiser, then the tensor-core GEMV")
                 del g
             del x_host, x_dev, y_dev, ys
         # Prefill T = 1024: act-quant + GEMM per shape (layer 0's weights).
@@ -861,6 +865,8 @@ def run_case(args):
     torch.cuda.set_device(dev)
     o, k = args.rows, args.cols
     vec = args.case in ("gemv", "linear", "seq")
+    if args.case == "step":
+        args.copies = 1
     copies = args.copies if vec else 1
     ws = build_weights(b, torch, dev, copies, [("w", o, k)], 6)
     T = args.batch if vec else args.tokens
@@ -869,7 +875,20 @@ def run_case(args):
     s = torch.empty(T, dtype=torch.float32, device=dev)
     y = torch.empty(copies * T * o, dtype=torch.float32, device=dev)
     b.bitnet_quant_act(x, T, k, q, s)
-    if args.case == "seq":
+    if args.case == "step":
+        # The benchmark's step: 30 BitNet-2B-shaped layers, one sequence call.
+        ws2 = build_weights(b, torch, dev, LAYERS, SHAPES, CONFIG_ID)
+        xh, xd, xv = make_inputs(torch, dev, LAYERS, SHAPES, 1, CONFIG_ID)
+        yd = torch.empty(sum(o_ for _, o_, _ in SHAPES) * LAYERS, dtype=torch.float32, device=dev)
+        ys2, off = [], 0
+        for l in range(LAYERS):
+            for _, o_, _ in SHAPES:
+                ys2.append(yd[off:off + o_])
+                off += o_
+        ents = linear_entries(ws2, LAYERS, SHAPES, xd, xv, ys2)
+        calls = [lambda: b.bitnet_w2a8_linear_seq(ents)]
+        copies = 1
+    elif args.case == "seq":
         ents = [(ws[(c, "w")], x[:k], y[c * o:(c + 1) * o], -1) for c in range(copies)]
         calls = [lambda: b.bitnet_w2a8_linear_seq(ents)]
     elif args.case == "linear":
@@ -893,7 +912,10 @@ def run_case(args):
     assert b.bitnet_get_device_error() == b.BITNET_OK
     med = sorted(times)[len(times) // 2]
     out = {"case": args.case, "out": o, "K": k, "T": T, "copies": copies, "us_per_linear": round(med, 3)}
-    if vec:
+    if args.case == "step":
+        out = {"case": "step", "us_per_step": round(med, 3),
+               "GB/s": round(fused_step_bytes() / (med * 1e-6) / 1e9, 1)}
+    elif vec:
         nbytes = gemv_bytes(o, k, T) if args.case == "gemv" else linear_bytes(o, k, T)
         out["GB/s"] = round(nbytes / (med * 1e-6) / 1e9, 1)
     elif args.case == "quant":
@@ -912,7 +934,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--case", choices=["gemv", "linear", "gemm", "quant", "seq"], help="profile one kernel on one shape")
+    ap.add_argument("--case", choices=["gemv", "linear", "gemm", "quant", "seq", "step"],
+                    help="profile one kernel on one shape (step: the benchmark's sequence call)")
     ap.add_argument("--rows", type=int, default=13824)
     ap.add_argument("--cols", type=int, default=2560)
     ap.add_argument("--batch", type=int, default=1)

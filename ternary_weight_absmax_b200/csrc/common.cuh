@@ -95,7 +95,7 @@ cudaError_t launch_ternarize(const float *w, int64_t rows, int64_t cols, bool pe
                              float *scales, double *partials, float *gamma_slot, cudaStream_t st);
 // Small-batch GEMV on the tensor cores (gemv_tc.cu): uniform rows, q and s
 // given, 1 <= B <= 64.
-constexpr int kTcMinBatch = 4;  // from this batch on the dispatcher prefers it to the dp4a kernels
+constexpr int kTcMinBatch = 8;  // from this batch on the dispatcher prefers it to the dp4a kernels (measured)
 bool gemv_tc_supported(int64_t rows, int64_t cols, int64_t B);
 cudaError_t launch_gemv_tc(const void *data, int64_t rows, int64_t cols, const int8_t *q, const float *s,
                            int64_t B, float *y, const DeviceGlobals &g, cudaStream_t st);

@@ -14,8 +14,8 @@ weights ("BitRun v0.2 实测：1-bit LLM 终端驾驶舱与毫瓦级功耗遥测
 Which kernel each case reaches (dispatch of the library, uniform rows):
   bitnet_w2a8_linear, B = 1, K <= 16384      -> batch-1 decode kernel, fused
   bitnet_w2a8_gemv,   B = 1, K <= 16384      -> batch-1 decode kernel
-  bitnet_w2a8_gemv,   B = 2, 3, K <= 16384   -> batched decode kernel
-  bitnet_w2a8_gemv,   B = 4..64              -> tensor-core kernel
+  bitnet_w2a8_gemv,   B = 2..7, K <= 16384   -> batched decode kernel
+  bitnet_w2a8_gemv,   B = 8..64              -> tensor-core kernel
   bitnet_w2a8_gemv_lut                       -> table-lookup kernel
   bitnet_w2a8_gemm                           -> tcgen05 GEMM, uniform path
 """

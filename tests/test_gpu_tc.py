@@ -1,6 +1,7 @@
-"""GPU parity of the small-batch paths for 4..64 tokens: the tensor-core GEMV
-(uniform rows; tcgen05 int8 MMA with the weights on the M side and K split
-over a cluster), the GEMM's block-scale path that bitnet_w2a8_gemv takes for
+"""GPU parity of the small-batch paths for 2..64 tokens: the batched dp4a
+decode kernel (2..7 tokens), the tensor-core GEMV (8..64 tokens, uniform rows;
+tcgen05 int8 MMA with the weights on the M side and K split over a cluster),
+the GEMM's block-scale path that bitnet_w2a8_gemv takes for
 17..64 tokens on per-block scales, and the two-kernel fused linear (quantiser
 into the caller's q_out / s_out, then the GEMV).  Against the oracle on the
 same seeded inputs: the int32 sums bit for bit (unit scales, s = 1), y within
@@ -48,7 +49,7 @@ SHAPES = [(1, 128), (17, 256), (128, 128), (129, 384), (777, 1280), (2560, 2560)
 
 
 @pytest.mark.parametrize("rows,K", SHAPES)
-@pytest.mark.parametrize("B", [4, 16, 17, 33, 64])
+@pytest.mark.parametrize("B", [4, 8, 16, 17, 33, 64])
 def test_tc_int32_sums_exact(rows, K, B):
     """Unit scales and integer activations with absmax 127 (s = 1): y is the
     exact int32 sum of every row and token."""
