@@ -359,16 +359,18 @@ __global__ void __launch_bounds__(kThreads, 1) decode_seq_kernel(const __grid_co
                 }
                 const int nt = min(kChunk, i1 - i);
                 const uint4 *wv = reinterpret_cast<const uint4 *>(ring + slot * (kChunk * kTile)) + lane;
-                if (nt == kChunk && j + kChunk < nb) {
-                    // A whole chunk inside the current row tile: no tile change.
+                for (int e = 0; e < nt;) {
+                    if (e + 4 <= nt && j + 4 < nb) {
+                        // Four items inside the current row tile: no tile change.
 #pragma unroll
-                    for (int e = 0; e < kChunk; e++) item(wv[e * 32], qp + e * 8);
-                    qp += kChunk * 8;
-                    j += kChunk;
-                } else {
-                    for (int e = 0; e < nt; e++) {
+                        for (int u = 0; u < 4; u++) item(wv[(e + u) * 32], qp + u * 8);
+                        qp += 32;
+                        j += 4;
+                        e += 4;
+                    } else {
                         item(wv[e * 32], qp);
                         qp += 8;
+                        e++;
                         if (++j == nb) {
                             flush();
                             r++;
