@@ -34,7 +34,7 @@
 //      tiles split between warps are summed in shared memory;
 //   C  the split tiles' rows are written; if a later linear reads this
 //      linear's y, the CTA adds its tile count to the linear's counter in the
-//      caller's workspace (after a fence), which the consumers poll (acquire)
+//      caller's workspace (a release add), which the consumers poll (acquire)
 //      until it reaches the linear's tile count.
 // Linears without a producer thus overlap freely (a CTA holds a contiguous
 // slice of the wave, usually one to three linears); a chain of dependent
@@ -230,7 +230,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_seq_kernel(const __grid_co
         const float ers = erow >= 0 ? __ldg(l.rowscale + erow) : 0.0f;
 
         // ---- A: producer, x, absmax, q, sum(q)
-        if (l.dep >= 0 && tid == 0) {
+        if (l.dep >= 0 && tid == 1) {
             // Each poll is an L2 round trip: a sixteenth of the copy-wait
             // iteration cap and the wall-clock cap bound the wait; another
             // CTA's abort ends it at once.
@@ -403,11 +403,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_seq_kernel(const __grid_co
             if (erow < l.rows && !*bad_w) l.y[erow] = __fmul_rn(__fmul_rn(ers, int_to_float(v - tot)), inv_s);
         }
         if (l.signal) {
+            // Every thread's y stores precede the barrier; one release add
+            // (cumulative over them) publishes the CTA's tiles.  Thread 1 does
+            // it: it issues no bulk copies, so nothing of its own is in flight.
             __syncthreads();
-            if (tid == 0 && !*bad_w) {
-                __threadfence();
-                atomicAdd(a.done + L, (unsigned)cnt);
-            }
+            if (tid == 1 && !*bad_w)
+                asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(a.done + L), "r"((unsigned)cnt)
+                             : "memory");
         }
     }
 

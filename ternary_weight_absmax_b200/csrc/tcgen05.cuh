@@ -39,32 +39,29 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
         : "memory");
     return ok != 0u;
 }
-// Nanosecond global timer.
-__device__ __forceinline__ uint64_t globaltimer_ns() {
-    uint64_t t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
-}
 // Wall-clock cap of every bounded wait: a try_wait may suspend the thread for
 // a system-dependent time, so an iteration cap alone does not bound the time.
-constexpr uint64_t kWaitCapNs = 2000000000ull;
+// Counted in SM cycles (clock64, a cheap register read; a %globaltimer read in
+// these loops measurably slowed the kernels that spin on mbarriers):
+// 4e9 cycles, about 2 s at the B200's clocks.
+constexpr long long kWaitCapCycles = 4000000000ll;
 
-// Tracks the wall-clock cap of one wait: checked every 64 tries.
+// Tracks the wall-clock cap of one wait: checked every 1024 tries.
 struct WaitClock {
-    uint64_t t0 = 0;
+    long long t0 = 0;
     __device__ __forceinline__ bool expired(uint32_t i) {
-        if ((i & 63u) != 63u) return false;
-        const uint64_t t = globaltimer_ns();
+        if ((i & 1023u) != 1023u) return false;
+        const long long t = clock64();
         if (t0 == 0) {
             t0 = t;
             return false;
         }
-        return t - t0 > kWaitCapNs;
+        return t - t0 > kWaitCapCycles;
     }
 };
 
 // Waits for the phase with the given parity to complete, at most `limit`
-// tries and about kWaitCapNs; gives up early once *abort is set.  Returns
+// tries and about kWaitCapCycles; gives up early once *abort is set.  Returns
 // false if it gave up.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint32_t limit,
                                           const volatile int *abort) {
