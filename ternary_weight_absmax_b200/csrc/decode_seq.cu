@@ -100,6 +100,21 @@ __device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned *p) {
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
 }
+// Wall-clock bound of the wait for a producer linear (polls of a global
+// counter, one L2 round trip each): 4e9 SM cycles, about 2 s, read every
+// 1024 polls.
+struct PollClock {
+    long long t0 = 0;
+    __device__ __forceinline__ bool expired(uint32_t i) {
+        if ((i & 1023u) != 1023u) return false;
+        const long long t = clock64();
+        if (t0 == 0) {
+            t0 = t;
+            return false;
+        }
+        return t - t0 > 4000000000ll;
+    }
+};
 __device__ __forceinline__ void prefetch_l2(const void *p) {
     asm volatile("prefetch.global.L2::evict_last [%0];" ::"l"(p));
 }
@@ -232,11 +247,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_seq_kernel(const __grid_co
         // ---- A: producer, x, absmax, q, sum(q)
         if (l.dep >= 0 && tid == 1) {
             // Each poll is an L2 round trip: a sixteenth of the copy-wait
-            // iteration cap and the wall-clock cap bound the wait; another
-            // CTA's abort ends it at once.
+            // iteration cap and a wall-clock cap bound the wait; another CTA's
+            // abort ends it at once.
             const uint32_t dlim = limit >> 4 ? limit >> 4 : 1u;
             uint32_t it = 0;
-            ptx::WaitClock clk;
+            PollClock clk;
             const unsigned need = (unsigned)a.lin[l.dep].ntr;
             while (ld_acquire_gpu(a.done + l.dep) < need) {
                 if (++it >= dlim || clk.expired(it) || *reinterpret_cast<volatile unsigned *>(a.abort)) {

@@ -39,37 +39,15 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
         : "memory");
     return ok != 0u;
 }
-// Wall-clock cap of every bounded wait: a try_wait may suspend the thread for
-// a system-dependent time, so an iteration cap alone does not bound the time.
-// Counted in SM cycles (clock64, a cheap register read; a %globaltimer read in
-// these loops measurably slowed the kernels that spin on mbarriers):
-// 4e9 cycles, about 2 s at the B200's clocks.
-constexpr long long kWaitCapCycles = 4000000000ll;
-
-// Tracks the wall-clock cap of one wait: checked every 1024 tries.
-struct WaitClock {
-    long long t0 = 0;
-    __device__ __forceinline__ bool expired(uint32_t i) {
-        if ((i & 1023u) != 1023u) return false;
-        const long long t = clock64();
-        if (t0 == 0) {
-            t0 = t;
-            return false;
-        }
-        return t - t0 > kWaitCapCycles;
-    }
-};
-
 // Waits for the phase with the given parity to complete, at most `limit`
-// tries and about kWaitCapCycles; gives up early once *abort is set.  Returns
-// false if it gave up.
+// tries; gives up early once *abort is set.  Returns false if it gave up.
+// (Adding a clock check to this loop, even one read every 1024 tries, slowed
+// the prefill GEMM from 100 to 174 us: the loop stays this minimal.)
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint32_t limit,
                                           const volatile int *abort) {
-    WaitClock clk;
     for (uint32_t i = 0; i < limit; i++) {
         if (mbar_try_wait(bar, parity)) return true;
         if (abort && *abort) return false;
-        if (clk.expired(i)) return false;
     }
     return false;
 }
@@ -97,11 +75,9 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *m, 
 // time (a whole main loop) so they do not take issue slots from busy warps.
 __device__ __forceinline__ bool mbar_wait_sleep(uint32_t bar, uint32_t parity, uint32_t limit,
                                                 const volatile int *abort, unsigned ns) {
-    WaitClock clk;
     for (uint32_t i = 0; i < limit; i++) {
         if (mbar_try_wait(bar, parity)) return true;
         if (abort && *abort) return false;
-        if (clk.expired(i)) return false;
         __nanosleep(ns);
     }
     return false;
