@@ -217,10 +217,11 @@ bitnet_status bitnet_quant_act(const float *x_dev, int64_t T, int64_t K, int8_t 
  *   - weights with uniform rows (BITNET_WEIGHT_UNIFORM_ROWS, the per-tensor
  *     absmean case): y = scale * acc * (1/s) in fp32 (three roundings, within
  *     2.4e-7 relative of the fp64 value), bit for bit the same for every B:
- *     B = 1 and K <= 16384 the batch-1 decode kernel (dp4a); B = 2..7 and
- *     K <= 16384 the batched decode kernel (dp4a); B >= 8 the tensor-core
- *     kernel (tcgen05 int8 MMA, weights on the M side, K split over a thread
- *     block cluster); otherwise the general kernel;
+ *     B = 1 and K <= 16384 the batch-1 decode kernel (dp4a); B = 2..4 and
+ *     K <= 16384 the batched decode kernel (dp4a); B >= 5 the tensor-core
+ *     kernel (warp-level int8 MMA, mma.sync m16n8k32, with the repacked code
+ *     tiles as its A fragments; K split over a thread block cluster);
+ *     otherwise the general kernel;
  *   - other weights: the sum over blocks runs in fp64 and is rounded once
  *     (the general kernel, exact for B <= 16; the GEMM's block-scale path,
  *     y = fp32(sum * (1/s)), for B > 16).
@@ -247,7 +248,7 @@ bitnet_status bitnet_w2a8_gemv(const bitnet_weight *w, const int8_t *q_dev, cons
  *   - With both (required for B > 16; q_out_dev then 16-byte aligned): the
  *     quantiser writes them, and the GEMV of bitnet_w2a8_gemv reads them (two
  *     kernels, the second overlapping its weight fetch with the first): the
- *     tensor-core kernel for uniform rows from B = 8 on.
+ *     tensor-core kernel for uniform rows from B = 5 on.
  * Errors: NULL (B > 16 without q_out_dev / s_out_dev), SHAPE, ALIGN, VALUE,
  * BUFSIZE, CUDA; BITNET_ERR_TIMEOUT is latched as for the GEMV. */
 bitnet_status bitnet_w2a8_linear(const bitnet_weight *w, const float *x_dev, int64_t B, float *y_dev,

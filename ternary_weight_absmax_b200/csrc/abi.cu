@@ -281,14 +281,14 @@ bitnet_status bitnet_quant_act(const float *x_dev, int64_t T, int64_t K, int8_t 
     return e == cudaSuccess ? BITNET_OK : cuda_fail(e, "quant_act launch");
 }
 
-// Device work of a GEMV on given q, s: the tensor-core kernel for uniform
-// rows from kTcMinBatch tokens, the decode / general kernels up to 16 tokens,
+// Device work of a GEMV on given q, s: the warp-MMA kernel for uniform rows
+// from kMmaMinBatch tokens, the decode / general kernels up to 16 tokens,
 // the GEMM's block-scale path (per-block fp64 sums) beyond.
 static cudaError_t gemv_dispatch(const bitnet_weight *w, const int8_t *q_dev, const float *s_dev, int64_t B,
                                  float *y_dev, int32_t *acc_dev, const DeviceGlobals &g, cudaStream_t st) {
     const bool uniform = (w->flags & BITNET_WEIGHT_UNIFORM_ROWS) != 0;
-    if (uniform && !acc_dev && B >= kTcMinBatch && gemv_tc_supported(w->rows, w->cols, B))
-        return launch_gemv_tc(w->data, w->rows, w->cols, q_dev, s_dev, B, y_dev, g, st);
+    if (uniform && !acc_dev && B >= kMmaMinBatch && gemv_mma_supported(w->rows, w->cols, B))
+        return launch_gemv_mma(w->data, w->rows, w->cols, q_dev, s_dev, B, y_dev, st);
     if (B <= 16)
         return launch_gemv(w->data, w->rows, w->cols, uniform, q_dev, s_dev, B, y_dev, acc_dev, nullptr, nullptr,
                            nullptr, g, st);

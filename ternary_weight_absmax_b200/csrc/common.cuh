@@ -93,12 +93,12 @@ cudaError_t launch_decode_lut(const void *data, int64_t rows, int64_t cols, cons
 int absmean_num_partials(int64_t n);
 cudaError_t launch_ternarize(const float *w, int64_t rows, int64_t cols, bool per_block, uint32_t *codes,
                              float *scales, double *partials, float *gamma_slot, cudaStream_t st);
-// Small-batch GEMV on the tensor cores (gemv_tc.cu): uniform rows, q and s
-// given, 1 <= B <= 64.
-constexpr int kTcMinBatch = 8;  // from this batch on the dispatcher prefers it to the dp4a kernels (measured)
-bool gemv_tc_supported(int64_t rows, int64_t cols, int64_t B);
-cudaError_t launch_gemv_tc(const void *data, int64_t rows, int64_t cols, const int8_t *q, const float *s,
-                           int64_t B, float *y, const DeviceGlobals &g, cudaStream_t st);
+// Small-batch GEMV on the warp-level int8 MMA (gemv_mma.cu): uniform rows, q
+// (16-byte aligned) and s given, 1 <= B <= 64.
+constexpr int kMmaMinBatch = 5;  // from this batch on the dispatcher prefers it to the dp4a kernels (measured)
+bool gemv_mma_supported(int64_t rows, int64_t cols, int64_t B);
+cudaError_t launch_gemv_mma(const void *data, int64_t rows, int64_t cols, const int8_t *q, const float *s,
+                            int64_t B, float *y, cudaStream_t st);
 // One linear of a sequence call (decode_seq.cu): repacked weight data with
 // uniform rows, fp32 x [cols], fp32 y [rows], and the index of the linear whose
 // y this x reads (-1: x is ready at launch).
