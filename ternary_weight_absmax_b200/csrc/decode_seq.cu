@@ -243,6 +243,22 @@ __global__ void __launch_bounds__(kThreads, 1) decode_seq_kernel(const __grid_co
             }
         }
         const float ers = erow >= 0 ? __ldg(l.rowscale + erow) : 0.0f;
+        // This warp's items and the row scales of its first tiles: they do not
+        // depend on a producer linear, so their loads overlap phase A (in a
+        // chain of dependent linears, each CTA's share of a linear is one or
+        // two tiles, and these loads were otherwise the first thing phase B
+        // waited for).
+        int i0, i1;
+        run_of(L, i0, i1);
+        float rsq[kRsDepth];
+        {
+            const int r = i0 / nb, rlast = (i1 - 1) / nb;
+#pragma unroll
+            for (int k = 0; k < kRsDepth; k++)
+                rsq[k] = i1 > i0 && r + k <= rlast
+                             ? __ldg(l.rowscale + (int64_t)(rlo + r + k) * kTileRows + (lane & 15))
+                             : 0.0f;
+        }
 
         // ---- A: producer, x, absmax, q, sum(q)
         if (l.dep >= 0 && tid == 1) {
@@ -305,18 +321,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_seq_kernel(const __grid_co
         if (tid == 0) *amax_w = 0u;  // every thread read it before (3)
 
         // ---- B: products over this warp's items [i0, i1)
-        int i0, i1;
-        run_of(L, i0, i1);
         if (ok && i1 > i0) {
             int r = i0 / nb, j = i0 - r * nb;
             const int rlast = (i1 - 1) / nb;
             const uint4 *qp = qrow + j * 8;
             int aA[4] = {0, 0, 0, 0}, aB[4] = {0, 0, 0, 0};
-            // Row scales of tiles r .. r + kRsDepth - 1 (lane l: row l & 15).
-            float rsq[kRsDepth];
-#pragma unroll
-            for (int k = 0; k < kRsDepth; k++)
-                rsq[k] = r + k <= rlast ? __ldg(l.rowscale + (int64_t)(rlo + r + k) * kTileRows + (lane & 15)) : 0.0f;
+            // rsq: row scales of tiles r .. r + kRsDepth - 1 (lane l: row l & 15).
             auto flush = [&]() {
                 const int pA = tig_reduce(combine4(aA));
                 const int pB = tig_reduce(combine4(aB));
