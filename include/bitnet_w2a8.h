@@ -272,6 +272,12 @@ bitnet_status bitnet_w2a8_linear(const bitnet_weight *w, const float *x_dev, int
  * (part of) the y of entry j, and this linear's products wait, on the device,
  * until every output of entry j is written.  Linears that wait for nothing
  * run concurrently; a chain of waits runs one linear after another.
+ * Performance note: each wait is a grid-wide hand-off through global memory
+ * (about 4.5 us per dependent linear on a B200, measured); for a pure chain
+ * (every entry waits for the one before it) one bitnet_w2a8_linear call per
+ * entry on one stream, whose kernels overlap their starts under programmatic
+ * dependent launch, is faster today (about 2.9 us per linear).  Lists whose
+ * entries are mostly independent of each other run fastest here.
  * Memory rules (checked on the host; BITNET_ERR_VALUE otherwise): no two y
  * ranges overlap, and an x range may overlap a y range only of an entry it
  * waits for directly or through a chain of waits, or of an entry that waits
