@@ -87,6 +87,10 @@ __device__ __forceinline__ void mma_u8s8(int (&d)[4], uint32_t a0, uint32_t a1, 
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// Bulk prefetch of `bytes` (a multiple of 16, 16-byte aligned) into L2.
+__device__ __forceinline__ void prefetch_l2_bulk(const void *p, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
 // Code words are read once: no L1 allocation, first out of L2.
 __device__ __forceinline__ uint4 ld_stream(const uint4 *p, uint64_t policy) {
     uint4 v;
@@ -110,34 +114,45 @@ __device__ __forceinline__ void cp_async_wait() {
     asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-// Gathers the activations of chunk `chunk` into buffer `buf` in fragment
-// order.  Region (block i, 8-token tile nt, half hf) of a chunk holds 128
-// words: word 4L + pos is lane L = 4g + t's B fragment register hb = pos & 1
-// of k slice grp = 2 hf + (pos >> 1), i.e. q[8 nt + g][128 j + 32 grp + 16 hb
-// + 4t .. + 3].  Thread `tid` copies word `tid` of every region (consecutive
-// threads, consecutive words: no bank conflicts).  Token rows past B are
-// never copied; the buffers are zeroed once.
+// Gathers the activations of a chunk into buffer `buf` in fragment order.
+// Region (block i, 8-token tile nt, half hf) of a chunk holds 128 words:
+// word 4L + pos is lane L = 4g + t's B fragment register hb = pos & 1 of k
+// slice grp = 2 hf + (pos >> 1), i.e. q[8 nt + g][128 j + 32 grp + 16 hb + 4t
+// .. + 3].  Thread `tid` copies word `tid` of every region (consecutive
+// threads, consecutive words: no bank conflicts); its source rows are fixed,
+// so their addresses are set up once (`Gather`).  Token rows past B are never
+// copied; the buffers are zeroed once.
 template <int NT>
-__device__ __forceinline__ void gather_chunk(const MmaArgs &a, uint32_t buf, int j0, int nj, int chunk, int tid) {
+struct Gather {
     using C = MmaCfg<NT>;
-    const int L = tid >> 2, pos = tid & 3, g = L >> 2, t = L & 3;
-    const int grp0 = pos >> 1, hb = pos & 1;
-#pragma unroll
-    for (int i = 0; i < C::kCH; i++) {
-        const int jj = chunk * C::kCH + i;
-        if (jj >= nj) break;
-        const int8_t *src = a.q + (int64_t)128 * (j0 + jj) + 32 * grp0 + 16 * hb + 4 * t;
+    const int8_t *src[C::kNTL];  // this thread's word of block 0, per 8-token tile (null past B)
+    __device__ __forceinline__ Gather(const MmaArgs &a, int j0, int tid) {
+        const int L = tid >> 2, pos = tid & 3, g = L >> 2, t = L & 3;
+        const int off = 128 * j0 + 32 * (pos >> 1) + 16 * (pos & 1) + 4 * t;
 #pragma unroll
         for (int nt = 0; nt < C::kNTL; nt++) {
             const int n = 8 * nt + g;
-            if (n < a.B) {
-                const uint32_t dst = buf + (uint32_t)(((i * C::kNTL + nt) * 2) * 512 + 4 * tid);
-                cp_async4(dst, src + (int64_t)n * a.cols);             // half 0: k slices 0, 1
-                cp_async4(dst + 512, src + (int64_t)n * a.cols + 64);  // half 1: k slices 2, 3
+            src[nt] = n < a.B ? a.q + (int64_t)n * a.cols + off : nullptr;
+        }
+    }
+    // Blocks chunk * kCH .. of the CTA's K slice (those below nj) into `buf`.
+    __device__ __forceinline__ void chunk(uint32_t buf, int nj, int chunk, int tid) const {
+#pragma unroll
+        for (int i = 0; i < C::kCH; i++) {
+            const int jj = chunk * C::kCH + i;
+            if (jj >= nj) break;
+#pragma unroll
+            for (int nt = 0; nt < C::kNTL; nt++) {
+                if (src[nt]) {
+                    const uint32_t dst = buf + (uint32_t)(((i * C::kNTL + nt) * 2) * 512 + 4 * tid);
+                    const int8_t *sp = src[nt] + 128 * jj;
+                    cp_async4(dst, sp);             // half 0: k slices 0, 1
+                    cp_async4(dst + 512, sp + 64);  // half 1: k slices 2, 3
+                }
             }
         }
     }
-}
+};
 
 template <int NT>
 __global__ void __launch_bounds__(kThreads, 4) gemv_mma_kernel(const MmaArgs a) {
@@ -166,6 +181,10 @@ __global__ void __launch_bounds__(kThreads, 4) gemv_mma_kernel(const MmaArgs a) 
 #pragma unroll
     for (int i = 0; i < PRE; i++)
         pre[i] = has_tile && i < nj ? ld_stream(cw + (int64_t)i * 32, policy) : make_uint4(0, 0, 0, 0);
+    // The rest of this warp's code words (one contiguous range of its tile)
+    // into L2 now: the register loads above keep only 4..8 K blocks in flight.
+    if (has_tile && lane == 0 && nj > PRE)
+        prefetch_l2_bulk(cw - lane + (int64_t)PRE * 32, (uint32_t)(nj - PRE) * kTileBytes);
     if (a.B < NT) {  // token rows past B stay zero in every activation buffer
         for (int i = threadIdx.x; i < C::kQD * C::kChunkBytes / 16; i += kThreads)
             reinterpret_cast<uint4 *>(smem)[i] = make_uint4(0, 0, 0, 0);
@@ -179,10 +198,11 @@ __global__ void __launch_bounds__(kThreads, 4) gemv_mma_kernel(const MmaArgs a) 
     }
     __syncthreads();  // the zero fill lands before the gathers
     const int nch = (nj + CH - 1) / CH;
+    const Gather<NT> gather(a, j0, threadIdx.x);
     // One cp.async group per activation chunk (empty past the last), kQD - 1 in flight.
 #pragma unroll
     for (int c = 0; c < C::kQD - 1; c++) {
-        if (c < nch) gather_chunk<NT>(a, sbase + (uint32_t)(c * C::kChunkBytes), j0, nj, c, threadIdx.x);
+        if (c < nch) gather.chunk(sbase + (uint32_t)(c * C::kChunkBytes), nj, c, threadIdx.x);
         cp_async_commit();
     }
     cp_async_wait<C::kQD - 2>();  // chunk 0 landed (this thread's copies)
@@ -205,7 +225,7 @@ __global__ void __launch_bounds__(kThreads, 4) gemv_mma_kernel(const MmaArgs a) 
     for (int c = 0; c < nch; c++) {
         // Buffer (c - 1) % kQD was last read by chunk c - 1, before the barrier.
         const int cn = c + C::kQD - 1;
-        if (cn < nch) gather_chunk<NT>(a, sbase + (uint32_t)((cn % C::kQD) * C::kChunkBytes), j0, nj, cn, threadIdx.x);
+        if (cn < nch) gather.chunk(sbase + (uint32_t)((cn % C::kQD) * C::kChunkBytes), nj, cn, threadIdx.x);
         cp_async_commit();
         const uint4 *qb = reinterpret_cast<const uint4 *>(smem + (c % C::kQD) * C::kChunkBytes) + lane;
 #pragma unroll
@@ -216,7 +236,19 @@ __global__ void __launch_bounds__(kThreads, 4) gemv_mma_kernel(const MmaArgs a) 
                 for (int nt = 0; nt < NTL; nt++) {
                     const uint4 h0 = qb[((i * NTL + nt) * 2 + 0) * 32];
                     const uint4 h1 = qb[((i * NTL + nt) * 2 + 1) * 32];
-                    if (has_tile) {
+                    if (has_tile && AS == 4) {
+                        // One set per k slice: the codes are masked in place
+                        // (bytes c * 4^(3 - grp) <= 128) and each set's sum is
+                        // shifted back after the loop, exactly.
+                        mma_u8s8(acc[0][nt], w.x & 0xC0C0C0C0u, w.y & 0xC0C0C0C0u, w.z & 0xC0C0C0C0u,
+                                 w.w & 0xC0C0C0C0u, h0.x, h0.y);
+                        mma_u8s8(acc[1 % AS][nt], w.x & 0x30303030u, w.y & 0x30303030u, w.z & 0x30303030u,
+                                 w.w & 0x30303030u, h0.z, h0.w);
+                        mma_u8s8(acc[2 % AS][nt], w.x & 0x0C0C0C0Cu, w.y & 0x0C0C0C0Cu, w.z & 0x0C0C0C0Cu,
+                                 w.w & 0x0C0C0C0Cu, h1.x, h1.y);
+                        mma_u8s8(acc[3 % AS][nt], w.x & 0x03030303u, w.y & 0x03030303u, w.z & 0x03030303u,
+                                 w.w & 0x03030303u, h1.z, h1.w);
+                    } else if (has_tile) {
                         mma_u8s8(acc[0][nt], (w.x >> 6) & 0x03030303u, (w.y >> 6) & 0x03030303u,
                                  (w.z >> 6) & 0x03030303u, (w.w >> 6) & 0x03030303u, h0.x, h0.y);
                         mma_u8s8(acc[1 % AS][nt], (w.x >> 4) & 0x03030303u, (w.y >> 4) & 0x03030303u,
@@ -253,6 +285,16 @@ __global__ void __launch_bounds__(kThreads, 4) gemv_mma_kernel(const MmaArgs a) 
         __syncthreads();
     }
     cp_async_wait<0>();
+    if (AS == 4) {  // undo the in-place scaling of the k slices' codes (exact shifts)
+#pragma unroll
+        for (int n = 0; n < NTL; n++)
+#pragma unroll
+            for (int i = 0; i < 4; i++) {
+                acc[0][n][i] >>= 6;
+                acc[1 % AS][n][i] >>= 4;
+                acc[2 % AS][n][i] >>= 2;
+            }
+    }
 #pragma unroll
     for (int u = 1; u < AS; u++)
 #pragma unroll
