@@ -78,9 +78,9 @@ struct SeqLin {
     const float *x;
     float *y;
     int64_t item_base;  // items of the earlier linears of the same wave
+    int64_t wave_items; // items of every linear of the same wave
     int ntr, nb, rows;
     int dep;            // index of the linear whose y this x reads, or -1
-    int wave;
     int signal;         // 1: a later linear waits for this one
 };
 
@@ -90,8 +90,7 @@ struct SeqArgs {
     unsigned *abort;       // set by a CTA that gave up, so the others stop waiting (workspace), or null
     unsigned *err;
     const unsigned *wait_limit;
-    int n, nwaves;
-    int64_t wave_items[kSeqMaxLinears];
+    int n;
     SeqLin lin[kSeqMaxLinears];
 };
 
@@ -137,17 +136,43 @@ __global__ void __launch_bounds__(kThreads, 1) decode_seq_kernel(const __grid_co
     const uint32_t bar0 = ptx::smem_u32(smem + kOffBar) + 8u * (warp * kSlots);
     const uint32_t limit = *a.wait_limit;
     const int n = a.n;
+    // The next kernel in the stream may start on the SMs this grid leaves;
+    // it reads nothing of ours before its own griddepcontrol.wait.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
-    // ---- this CTA's row tiles of every linear: [seg_lo, seg_lo + seg_cnt)
-    for (int L = tid; L < n; L += kThreads) {
-        const SeqLin &l = a.lin[L];
-        const int64_t W = a.wave_items[l.wave];
-        const int64_t lo = (int64_t)c * W / G - l.item_base;
-        const int64_t hi = (int64_t)(c + 1) * W / G - l.item_base;
-        const int64_t rlo = min((int64_t)l.ntr, lo <= 0 ? 0 : (lo + l.nb - 1) / l.nb);
-        const int64_t rhi = min((int64_t)l.ntr, hi <= 0 ? 0 : (hi + l.nb - 1) / l.nb);
-        seg_lo[L] = (int)rlo;
-        seg_cnt[L] = (int)(rhi - rlo);
+    // ---- this CTA's row tiles of every linear: [seg_lo, seg_lo + seg_cnt).
+    // The list sits in the kernel parameters, behind the constant cache, which
+    // serves the lanes of a warp that read different addresses one after
+    // another: with one linear per lane this loop took 8-16 us.  Here every
+    // lane of a warp reads the same linear, kPro linears per warp at a time
+    // (their loads independent, so in flight together), and lane u keeps
+    // linear u of the batch.
+    constexpr int kPro = 8;
+    for (int L0 = warp * kPro; L0 < n; L0 += kWarps * kPro) {
+        int64_t base = 0, W = 0;
+        int ntr = 0, nb = 1;
+#pragma unroll
+        for (int u = 0; u < kPro; u++) {
+            if (L0 + u < n) {
+                const SeqLin &l = a.lin[L0 + u];
+                const int64_t base_u = l.item_base, W_u = l.wave_items;
+                const int ntr_u = l.ntr, nb_u = l.nb;
+                if (lane == u) {
+                    base = base_u;
+                    W = W_u;
+                    ntr = ntr_u;
+                    nb = nb_u;
+                }
+            }
+        }
+        if (lane < kPro && L0 + lane < n) {
+            const int64_t lo = (int64_t)c * W / G - base;
+            const int64_t hi = (int64_t)(c + 1) * W / G - base;
+            const int64_t rlo = min((int64_t)ntr, lo <= 0 ? 0 : (lo + nb - 1) / nb);
+            const int64_t rhi = min((int64_t)ntr, hi <= 0 ? 0 : (hi + nb - 1) / nb);
+            seg_lo[L0 + lane] = (int)rlo;
+            seg_cnt[L0 + lane] = (int)(rhi - rlo);
+        }
     }
     for (int i = tid; i < kSmallTiles * kTileRows; i += kThreads) acc[i] = 0;
     if (tid == 0) {
@@ -209,10 +234,20 @@ __global__ void __launch_bounds__(kThreads, 1) decode_seq_kernel(const __grid_co
         ii += nt;
         if (ii >= iend) next_run();
     };
+    // The first segment's x into L2 ahead of the weight copies (a prefetch
+    // reads nothing into this SM, so it may precede griddepcontrol.wait).
+    if (nseg > 0 && a.lin[seg_list[0]].dep < 0) {
+        const SeqLin &l0 = a.lin[seg_list[0]];
+        for (int i = tid; i < l0.nb * 4; i += kThreads) prefetch_l2(l0.x + i * 32);
+    }
     if (lane == 0) {
         next_run();
         for (int k = 0; k < kSlots; k++) issue();
     }
+    // Weights are never written by a kernel, so their copies start before the
+    // wait for the previous kernel in the stream (programmatic dependent
+    // launch); x, y and the workspace counters are touched only after it.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 
     uint32_t cq = 0;                      // chunks consumed (every lane keeps the same count)
     uint32_t cslot = 0, cphase = 0;       // its slot and the parity of that slot's phase
@@ -480,6 +515,7 @@ cudaError_t launch_decode_seq(const SeqLinear *list, int n, void *workspace, con
     a.n = n;
     // Waves: 0 without a producer, else one more than the producer's.
     int wave[kSeqMaxLinears];
+    int64_t wave_items[kSeqMaxLinears];
     int nwaves = 0;
     bool any_dep = false;
     for (int i = 0; i < n; i++) {
@@ -487,8 +523,7 @@ cudaError_t launch_decode_seq(const SeqLinear *list, int n, void *workspace, con
         nwaves = wave[i] + 1 > nwaves ? wave[i] + 1 : nwaves;
         any_dep = any_dep || list[i].dep >= 0;
     }
-    a.nwaves = nwaves;
-    for (int w = 0; w < nwaves; w++) a.wave_items[w] = 0;
+    for (int w = 0; w < nwaves; w++) wave_items[w] = 0;
     for (int i = 0; i < n; i++) {
         const Layout Lo = layout_of(list[i].rows, list[i].cols);
         const unsigned char *base = static_cast<const unsigned char *>(list[i].data);
@@ -501,11 +536,11 @@ cudaError_t launch_decode_seq(const SeqLinear *list, int n, void *workspace, con
         l.nb = (int)Lo.nb;
         l.rows = (int)list[i].rows;
         l.dep = list[i].dep;
-        l.wave = wave[i];
         l.signal = 0;
-        l.item_base = a.wave_items[wave[i]];
-        a.wave_items[wave[i]] += (int64_t)Lo.ntr * Lo.nb;
+        l.item_base = wave_items[wave[i]];
+        wave_items[wave[i]] += (int64_t)Lo.ntr * Lo.nb;
     }
+    for (int i = 0; i < n; i++) a.lin[i].wave_items = wave_items[wave[i]];
     for (int i = 0; i < n; i++)
         if (list[i].dep >= 0) a.lin[list[i].dep].signal = 1;
     unsigned *ws = static_cast<unsigned *>(workspace);
@@ -521,8 +556,14 @@ cudaError_t launch_decode_seq(const SeqLinear *list, int n, void *workspace, con
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeCooperative;  // producer waits need every CTA resident
     attr[0].val.cooperative = 1;
+    if (!any_dep) {
+        // Without producer waits: programmatic dependent launch, so the
+        // prologue and the first weight copies overlap the previous kernel.
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+    }
     cfg.attrs = attr;
-    cfg.numAttrs = any_dep ? 1 : 0;
+    cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, decode_seq_kernel, a);
 }
 
