@@ -290,7 +290,11 @@ bitnet_status bitnet_w2a8_linear(const bitnet_weight *w, const float *x_dev, int
  * may be NULL (and workspace_bytes 0) when no entry waits.  Calls that share
  * a workspace must not overlap on the GPU.  A call with waits is a
  * cooperative launch (one CTA per SM, all resident); it fails with
- * BITNET_ERR_CUDA if the device cannot co-schedule them.
+ * BITNET_ERR_CUDA if the device cannot co-schedule them.  A call without
+ * waits is a programmatic dependent launch: its set-up and first weight
+ * copies may start while the previous kernel on `stream` finishes, and it
+ * reads x, writes y and touches the workspace only after that kernel is
+ * complete, so stream order holds as for any launch.
  * Errors: NULL, SHAPE (n outside 1..BITNET_SEQ_MAX_LINEARS), ALIGN, VALUE
  * (bad wait_for, not repacked, overlapping buffers), UNSUPPORTED (rows not
  * uniform, or cols > BITNET_SEQ_MAX_COLS), BUFSIZE (workspace), CUDA.  Bounded
