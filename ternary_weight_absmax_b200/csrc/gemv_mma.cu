@@ -40,9 +40,14 @@
 // conflict-free 16-byte loads) with 4-byte cp.async copies, three chunks
 // ahead.  sum q of each token over the CTA's K slice is taken with dp4a from
 // the B fragments the warps load anyway, each (block, 8-token tile) by one
-// warp.  The only waits are CTA and cluster barriers.  (A version that
-// streamed the code words through per-warp bulk-copy rings in shared memory
-// measured the same to 50% slower, depending on the shape.)
+// warp.  The only waits are CTA and cluster barriers.  A grid that fits in
+// three CTAs per SM asks for enough shared memory that no SM holds a fourth:
+// under programmatic dependent launch the CTAs start on the SMs the previous
+// kernel leaves first, and without the cap they piled up four to an SM while
+// other SMs stayed empty (16 tokens on 20480 x 3200: 13.8 -> 12.3 us; with the
+// code-word registers used in rotating groups rather than shifted: 11.4 us).
+// (A version that streamed the code words through per-warp bulk-copy rings in
+// shared memory measured the same to 50% slower, depending on the shape.)
 #include <atomic>
 
 #include "common.cuh"
@@ -176,7 +181,7 @@ __global__ void __launch_bounds__(kThreads, 4) gemv_mma_kernel(const MmaArgs a) 
 
     // The first code words: weights do not depend on the previous kernel.
     constexpr int PRE = C::kPre;
-    static_assert(PRE % CH == 0, "code words move down a chunk at a time");
+    static_assert(PRE % CH == 0, "code words are held in whole chunks");
     uint4 pre[PRE];
 #pragma unroll
     for (int i = 0; i < PRE; i++)
@@ -222,67 +227,72 @@ __global__ void __launch_bounds__(kThreads, 4) gemv_mma_kernel(const MmaArgs a) 
             for (int i = 0; i < 4; i++) acc[u][n][i] = 0;
     }
 
-    for (int c = 0; c < nch; c++) {
-        // Buffer (c - 1) % kQD was last read by chunk c - 1, before the barrier.
-        const int cn = c + C::kQD - 1;
-        if (cn < nch) gather.chunk(sbase + (uint32_t)((cn % C::kQD) * C::kChunkBytes), nj, cn, threadIdx.x);
-        cp_async_commit();
-        const uint4 *qb = reinterpret_cast<const uint4 *>(smem + (c % C::kQD) * C::kChunkBytes) + lane;
+    // The code words of chunk c sit in register group c % M (M = PRE / CH);
+    // once used, the group is refilled with chunk c + M.  Unrolled over the
+    // groups so that no word moves between registers.
+    constexpr int M = PRE / CH;
+#pragma unroll 1
+    for (int c0 = 0; c0 < nch; c0 += M) {
 #pragma unroll
-        for (int i = 0; i < CH; i++) {
-            if (c * CH + i < nj) {
-                const uint4 w = pre[i];
+        for (int u = 0; u < M; u++) {
+            const int c = c0 + u;
+            if (c >= nch) break;
+            const int cn = c + C::kQD - 1;
+            if (cn < nch) gather.chunk(sbase + (uint32_t)((cn % C::kQD) * C::kChunkBytes), nj, cn, threadIdx.x);
+            cp_async_commit();
+            const uint4 *qb = reinterpret_cast<const uint4 *>(smem + (c % C::kQD) * C::kChunkBytes) + lane;
 #pragma unroll
-                for (int nt = 0; nt < NTL; nt++) {
-                    const uint4 h0 = qb[((i * NTL + nt) * 2 + 0) * 32];
-                    const uint4 h1 = qb[((i * NTL + nt) * 2 + 1) * 32];
-                    if (has_tile && AS == 4) {
-                        // One set per k slice: the codes are masked in place
-                        // (bytes c * 4^(3 - grp) <= 128) and each set's sum is
-                        // shifted back after the loop, exactly.
-                        mma_u8s8(acc[0][nt], w.x & 0xC0C0C0C0u, w.y & 0xC0C0C0C0u, w.z & 0xC0C0C0C0u,
-                                 w.w & 0xC0C0C0C0u, h0.x, h0.y);
-                        mma_u8s8(acc[1 % AS][nt], w.x & 0x30303030u, w.y & 0x30303030u, w.z & 0x30303030u,
-                                 w.w & 0x30303030u, h0.z, h0.w);
-                        mma_u8s8(acc[2 % AS][nt], w.x & 0x0C0C0C0Cu, w.y & 0x0C0C0C0Cu, w.z & 0x0C0C0C0Cu,
-                                 w.w & 0x0C0C0C0Cu, h1.x, h1.y);
-                        mma_u8s8(acc[3 % AS][nt], w.x & 0x03030303u, w.y & 0x03030303u, w.z & 0x03030303u,
-                                 w.w & 0x03030303u, h1.z, h1.w);
-                    } else if (has_tile) {
-                        mma_u8s8(acc[0][nt], (w.x >> 6) & 0x03030303u, (w.y >> 6) & 0x03030303u,
-                                 (w.z >> 6) & 0x03030303u, (w.w >> 6) & 0x03030303u, h0.x, h0.y);
-                        mma_u8s8(acc[1 % AS][nt], (w.x >> 4) & 0x03030303u, (w.y >> 4) & 0x03030303u,
-                                 (w.z >> 4) & 0x03030303u, (w.w >> 4) & 0x03030303u, h0.z, h0.w);
-                        mma_u8s8(acc[2 % AS][nt], (w.x >> 2) & 0x03030303u, (w.y >> 2) & 0x03030303u,
-                                 (w.z >> 2) & 0x03030303u, (w.w >> 2) & 0x03030303u, h1.x, h1.y);
-                        mma_u8s8(acc[3 % AS][nt], w.x & 0x03030303u, w.y & 0x03030303u, w.z & 0x03030303u,
-                                 w.w & 0x03030303u, h1.z, h1.w);
-                    }
-                    if ((i * NTL + nt) % kWarps == warp) {  // this warp's share of sum q
-                        int v = __dp4a((int)h0.x, 0x01010101, sqp[nt]);
-                        v = __dp4a((int)h0.y, 0x01010101, v);
-                        v = __dp4a((int)h0.z, 0x01010101, v);
-                        v = __dp4a((int)h0.w, 0x01010101, v);
-                        v = __dp4a((int)h1.x, 0x01010101, v);
-                        v = __dp4a((int)h1.y, 0x01010101, v);
-                        v = __dp4a((int)h1.z, 0x01010101, v);
-                        sqp[nt] = __dp4a((int)h1.w, 0x01010101, v);
+            for (int i = 0; i < CH; i++) {
+                if (c * CH + i < nj) {
+                    const uint4 w = pre[u * CH + i];
+#pragma unroll
+                    for (int nt = 0; nt < NTL; nt++) {
+                        const uint4 h0 = qb[((i * NTL + nt) * 2 + 0) * 32];
+                        const uint4 h1 = qb[((i * NTL + nt) * 2 + 1) * 32];
+                        if (has_tile && AS == 4) {
+                            // One set per k slice: the codes are masked in place
+                            // (bytes c * 4^(3 - grp) <= 128) and each set's sum is
+                            // shifted back after the loop, exactly.
+                            mma_u8s8(acc[0][nt], w.x & 0xC0C0C0C0u, w.y & 0xC0C0C0C0u, w.z & 0xC0C0C0C0u,
+                                     w.w & 0xC0C0C0C0u, h0.x, h0.y);
+                            mma_u8s8(acc[1 % AS][nt], w.x & 0x30303030u, w.y & 0x30303030u, w.z & 0x30303030u,
+                                     w.w & 0x30303030u, h0.z, h0.w);
+                            mma_u8s8(acc[2 % AS][nt], w.x & 0x0C0C0C0Cu, w.y & 0x0C0C0C0Cu, w.z & 0x0C0C0C0Cu,
+                                     w.w & 0x0C0C0C0Cu, h1.x, h1.y);
+                            mma_u8s8(acc[3 % AS][nt], w.x & 0x03030303u, w.y & 0x03030303u, w.z & 0x03030303u,
+                                     w.w & 0x03030303u, h1.z, h1.w);
+                        } else if (has_tile) {
+                            mma_u8s8(acc[0][nt], (w.x >> 6) & 0x03030303u, (w.y >> 6) & 0x03030303u,
+                                     (w.z >> 6) & 0x03030303u, (w.w >> 6) & 0x03030303u, h0.x, h0.y);
+                            mma_u8s8(acc[1 % AS][nt], (w.x >> 4) & 0x03030303u, (w.y >> 4) & 0x03030303u,
+                                     (w.z >> 4) & 0x03030303u, (w.w >> 4) & 0x03030303u, h0.z, h0.w);
+                            mma_u8s8(acc[2 % AS][nt], (w.x >> 2) & 0x03030303u, (w.y >> 2) & 0x03030303u,
+                                     (w.z >> 2) & 0x03030303u, (w.w >> 2) & 0x03030303u, h1.x, h1.y);
+                            mma_u8s8(acc[3 % AS][nt], w.x & 0x03030303u, w.y & 0x03030303u, w.z & 0x03030303u,
+                                     w.w & 0x03030303u, h1.z, h1.w);
+                        }
+                        if ((i * NTL + nt) % kWarps == warp) {  // this warp's share of sum q
+                            int v = __dp4a((int)h0.x, 0x01010101, sqp[nt]);
+                            v = __dp4a((int)h0.y, 0x01010101, v);
+                            v = __dp4a((int)h0.z, 0x01010101, v);
+                            v = __dp4a((int)h0.w, 0x01010101, v);
+                            v = __dp4a((int)h1.x, 0x01010101, v);
+                            v = __dp4a((int)h1.y, 0x01010101, v);
+                            v = __dp4a((int)h1.z, 0x01010101, v);
+                            sqp[nt] = __dp4a((int)h1.w, 0x01010101, v);
+                        }
                     }
                 }
             }
-        }
-        // Next code words: the held ones move down a chunk, one chunk is fetched.
 #pragma unroll
-        for (int i = 0; i < PRE; i++) {
-            if (i + CH < PRE) {
-                pre[i] = pre[i + CH];
-            } else {
-                const int jj = (c + 1) * CH + i;
-                pre[i] = has_tile && jj < nj ? ld_stream(cw + (int64_t)jj * 32, policy) : make_uint4(0, 0, 0, 0);
+            for (int i = 0; i < CH; i++) {
+                const int jj = (c + M) * CH + i;
+                pre[u * CH + i] =
+                    has_tile && jj < nj ? ld_stream(cw + (int64_t)jj * 32, policy) : make_uint4(0, 0, 0, 0);
             }
+            cp_async_wait<C::kQD - 2>();  // chunk c + 1 landed
+            __syncthreads();
         }
-        cp_async_wait<C::kQD - 2>();  // chunk c + 1 landed
-        __syncthreads();
     }
     cp_async_wait<0>();
     if (AS == 4) {  // undo the in-place scaling of the k slices' codes (exact shifts)
@@ -369,14 +379,17 @@ cudaError_t run_mma(const MmaArgs &a, int64_t mtiles, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     if (!configured[dev].load(std::memory_order_acquire)) {
-        e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::kSmem);
+        e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, 60 * 1024);
         if (e != cudaSuccess) return e;
         configured[dev].store(true, std::memory_order_release);
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(mtiles * a.splits));
     cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = C::kSmem;
+    // A grid that fits in three CTAs per SM asks for enough shared memory
+    // that no SM takes a fourth: when the previous kernel's CTAs leave the
+    // SMs one by one, this spreads the CTAs over more SMs.
+    cfg.dynamicSmemBytes = mtiles * a.splits <= 3 * (int64_t)num_sms() ? 60 * 1024 : C::kSmem;
     cfg.stream = st;
     cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
