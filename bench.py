@@ -573,25 +573,36 @@ def run_llama8b(b, torch, dev, T, peaks):
 
 
 def prefill_shapes(b, torch, dev, T, peaks, cases, tokens):
+    """Per shape: bitnet_w2a8_gemm (weights decoded in the kernel, per
+    128-token tile), bitnet_w2a8_gemm_ws (weights expanded to int8 once per
+    call, then the pair-of-SMs GEMM), the quantiser, and the quantiser
+    followed by each GEMM (the prefill linear, x fp32 -> y)."""
     out = {}
     for name, o, k, w in cases:
         x = torch.randn(tokens * k, dtype=torch.float32, device=dev)
         q = torch.empty(tokens * k, dtype=torch.int8, device=dev)
         s = torch.empty(tokens, dtype=torch.float32, device=dev)
         y = torch.empty(tokens * o, dtype=torch.float32, device=dev)
+        ws = torch.empty(b.bitnet_w2a8_gemm_workspace_bytes(o, k), dtype=torch.uint8, device=dev)
         g_q = T.capture(lambda: b.bitnet_quant_act(x, tokens, k, q, s))
         g_m = T.capture(lambda: b.bitnet_w2a8_gemm(w, q, s, tokens, y))
+        g_w = T.capture(lambda: b.bitnet_w2a8_gemm_ws(w, q, s, tokens, y, ws))
         g_b = T.capture(lambda: (b.bitnet_quant_act(x, tokens, k, q, s), b.bitnet_w2a8_gemm(w, q, s, tokens, y)))
-        mq, mm, mb = T.ms(g_q, 10), T.ms(g_m, 10), T.ms(g_b, 10)
+        g_bw = T.capture(lambda: (b.bitnet_quant_act(x, tokens, k, q, s),
+                                  b.bitnet_w2a8_gemm_ws(w, q, s, tokens, y, ws)))
+        mq, mm, mw, mb, mbw = T.ms(g_q, 10), T.ms(g_m, 10), T.ms(g_w, 10), T.ms(g_b, 10), T.ms(g_bw, 10)
         ops = 2.0 * tokens * o * k
         tops = ops / (mm * 1e-3) / 1e12
+        tops_w = ops / (mw * 1e-3) / 1e12
         qbytes = 4 * tokens * k + tokens * k + 4 * tokens
         out[name] = {"out": o, "K": k, "T": tokens, "gemm_us": round(mm * 1e3, 2), "TOPS": round(tops, 1),
                      "frac_of_int8_peak": round(tops / peaks["int8_tops"], 4),
+                     "gemm_ws_us": round(mw * 1e3, 2), "ws_TOPS": round(tops_w, 1),
+                     "ws_frac_of_int8_peak": round(tops_w / peaks["int8_tops"], 4),
                      "act_quant_us": round(mq * 1e3, 2),
                      "act_quant_GB/s": round(qbytes / (mq * 1e-3) / 1e9, 1),
-                     "linear_us": round(mb * 1e3, 2)}
-        del g_q, g_m, g_b
+                     "linear_us": round(mb * 1e3, 2), "linear_ws_us": round(mbw * 1e3, 2)}
+        del g_q, g_m, g_w, g_b, g_bw, ws
     return out
 
 
@@ -602,7 +613,7 @@ def run_prefill(b, torch, dev, T, peaks):
         for tokens in (512, 2048):
             res[f"T{tokens}"] = prefill_shapes(b, torch, dev, T, peaks,
                                                [(n, o, k, weights[(0, n)]) for n, o, k in PREFILL], tokens)
-        best = max(v["TOPS"] for tt in ("T512", "T2048") for v in res[tt].values())
+        best = max(max(v["TOPS"], v["ws_TOPS"]) for tt in ("T512", "T2048") for v in res[tt].values())
         res["best_frac_of_int8_peak"] = round(best / peaks["int8_tops"], 4)
         del weights
     except Exception as e:  # reported beside the headline, never instead of it

@@ -323,6 +323,25 @@ bitnet_status bitnet_w2a8_linear_seq(const bitnet_linear_desc *list, int32_t n, 
 bitnet_status bitnet_w2a8_gemm(const bitnet_weight *w, const int8_t *q_dev, const float *s_dev,
                                int64_t T, float *y_dev, bitnet_stream_t stream);
 
+/* The same GEMM with a caller-owned workspace for the weights expanded to
+ * int8.  On uniform rows from 256 tokens the call first expands the packed
+ * codes to t = c - 1 bytes, [rows rounded up to 16][cols] row-major, in the
+ * workspace (one pass, 4 bytes written per packed byte read), then runs the
+ * tcgen05 GEMM with both operands loaded by TMA: each weight is decoded once
+ * per call instead of once per 128-token tile.  Same y, bit for bit, as
+ * bitnet_w2a8_gemm.  Below 256 tokens, on block-scale weights, or with
+ * workspace_dev NULL it is bitnet_w2a8_gemm.
+ * workspace_dev: device memory of at least
+ * bitnet_w2a8_gemm_workspace_bytes(rows, cols) bytes, 256-byte aligned,
+ * caller owned, contents undefined between calls; calls that share it must
+ * be stream ordered (the expansion waits for the previous kernel on `stream`
+ * before it writes).  Errors: those of bitnet_w2a8_gemm, ALIGN (workspace),
+ * BUFSIZE (workspace too small). */
+size_t bitnet_w2a8_gemm_workspace_bytes(int64_t rows, int64_t cols);
+bitnet_status bitnet_w2a8_gemm_ws(const bitnet_weight *w, const int8_t *q_dev, const float *s_dev, int64_t T,
+                                  float *y_dev, void *workspace_dev, size_t workspace_bytes,
+                                  bitnet_stream_t stream);
+
 /* Table-lookup variant of bitnet_w2a8_gemv at B = 1, kept for comparison with
  * the dp4a kernels: the CPU kernels of "浏览器里跑 1-bit 大模型 BitNet
  * WebAssembly 的 50 倍提速实操" (section "查表（LUT）内核") replace products by

@@ -85,6 +85,8 @@ def _load() -> ctypes.CDLL:
         "bitnet_quant_act": ([vp, i64, i64, vp, vp, vp, vp], st),
         "bitnet_w2a8_gemv": ([W, vp, vp, i64, vp, vp], st),
         "bitnet_w2a8_gemm": ([W, vp, vp, i64, vp, vp], st),
+        "bitnet_w2a8_gemm_workspace_bytes": ([i64, i64], sz),
+        "bitnet_w2a8_gemm_ws": ([W, vp, vp, i64, vp, vp, sz, vp], st),
         "bitnet_w2a8_linear": ([W, vp, i64, vp, vp, vp, vp], st),
         "bitnet_w2a8_linear_acc": ([W, vp, i64, vp, vp, vp, vp, vp], st),
         "bitnet_w2a8_gemv_acc": ([W, vp, vp, i64, vp, vp, vp], st),
@@ -269,6 +271,21 @@ def bitnet_w2a8_gemv(w: Weight, q, s, B: int, y, stream=None):
 def bitnet_w2a8_gemm(w: Weight, q, s, T: int, y, stream=None):
     _check(_lib.bitnet_w2a8_gemm(w.ref(), _dptr(q, "int8", T * w.cols, "q"), _dptr(s, "float32", T, "s"), T,
                                  _dptr(y, "float32", T * w.rows, "y"), _stream(stream)), "bitnet_w2a8_gemm")
+
+
+def bitnet_w2a8_gemm_workspace_bytes(rows: int, cols: int) -> int:
+    return _lib.bitnet_w2a8_gemm_workspace_bytes(rows, cols)
+
+
+def bitnet_w2a8_gemm_ws(w: Weight, q, s, T: int, y, workspace, stream=None):
+    """bitnet_w2a8_gemm with a workspace (uint8 CUDA tensor of
+    bitnet_w2a8_gemm_workspace_bytes(rows, cols) bytes, or None)."""
+    n = bitnet_w2a8_gemm_workspace_bytes(w.rows, w.cols)
+    ws = _dptr(workspace, "uint8", n, "workspace") if workspace is not None else None
+    _check(_lib.bitnet_w2a8_gemm_ws(w.ref(), _dptr(q, "int8", T * w.cols, "q"), _dptr(s, "float32", T, "s"), T,
+                                    _dptr(y, "float32", T * w.rows, "y"), ws,
+                                    workspace.numel() if workspace is not None else 0, _stream(stream)),
+           "bitnet_w2a8_gemm_ws")
 
 
 def bitnet_w2a8_linear(w: Weight, x, B: int, y, q_out=None, s_out=None, stream=None):

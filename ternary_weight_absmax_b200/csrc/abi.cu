@@ -447,7 +447,8 @@ bitnet_status bitnet_w2a8_linear_seq(const bitnet_linear_desc *list, int32_t n, 
 }
 
 static bitnet_status gemm_impl(const bitnet_weight *w, const int8_t *q_dev, const float *s_dev,
-                               int64_t T, float *y_dev, int32_t *acc_dev, bitnet_stream_t stream) {
+                               int64_t T, float *y_dev, int32_t *acc_dev, bitnet_stream_t stream,
+                               void *workspace_dev = nullptr, size_t workspace_bytes = 0) {
     t_detail[0] = 0;
     bitnet_status s = check_weight(w);
     if (s != BITNET_OK) return s;
@@ -456,6 +457,12 @@ static bitnet_status gemm_impl(const bitnet_weight *w, const int8_t *q_dev, cons
     if (!q_dev || !s_dev || !y_dev) return fail(BITNET_ERR_NULL, "NULL pointer");
     if (!aligned(q_dev, 16) || !aligned(s_dev, 4) || !aligned(y_dev, 16) || (acc_dev && !aligned(acc_dev, 4)))
         return fail(BITNET_ERR_ALIGN, "q and y need 16-byte, s/acc 4-byte alignment");
+    if (workspace_dev) {
+        if (!aligned(workspace_dev, 256)) return fail(BITNET_ERR_ALIGN, "workspace needs 256-byte alignment");
+        if (workspace_bytes < gemm_expanded_bytes(w->rows, w->cols))
+            return fail(BITNET_ERR_BUFSIZE, "workspace %zu < %zu bytes", workspace_bytes,
+                        gemm_expanded_bytes(w->rows, w->cols));
+    }
     int dev = 0, major = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
@@ -465,13 +472,25 @@ static bitnet_status gemm_impl(const bitnet_weight *w, const int8_t *q_dev, cons
     e = device_globals(&g);
     if (e != cudaSuccess) return cuda_fail(e, "device globals");
     e = launch_gemm(w->data, w->rows, w->cols, (w->flags & BITNET_WEIGHT_UNIFORM_ROWS) != 0, q_dev, s_dev,
-                    T, y_dev, acc_dev, g, reinterpret_cast<cudaStream_t>(stream));
+                    T, y_dev, acc_dev, g, reinterpret_cast<cudaStream_t>(stream),
+                    static_cast<int8_t *>(workspace_dev));
     return e == cudaSuccess ? BITNET_OK : cuda_fail(e, "gemm launch");
 }
 
 bitnet_status bitnet_w2a8_gemm(const bitnet_weight *w, const int8_t *q_dev, const float *s_dev, int64_t T,
                                float *y_dev, bitnet_stream_t stream) {
     return gemm_impl(w, q_dev, s_dev, T, y_dev, nullptr, stream);
+}
+
+size_t bitnet_w2a8_gemm_workspace_bytes(int64_t rows, int64_t cols) {
+    if (rows < 1 || cols < kQK || cols % kQK != 0 || rows > kMaxRows || cols > kMaxCols) return 0;
+    return gemm_expanded_bytes(rows, cols);
+}
+
+bitnet_status bitnet_w2a8_gemm_ws(const bitnet_weight *w, const int8_t *q_dev, const float *s_dev, int64_t T,
+                                  float *y_dev, void *workspace_dev, size_t workspace_bytes,
+                                  bitnet_stream_t stream) {
+    return gemm_impl(w, q_dev, s_dev, T, y_dev, nullptr, stream, workspace_dev, workspace_bytes);
 }
 
 bitnet_status bitnet_w2a8_gemm_acc(const bitnet_weight *w, const int8_t *q_dev, const float *s_dev,

@@ -114,8 +114,19 @@ struct SeqLinear {
 size_t seq_workspace_bytes(int n);
 cudaError_t launch_decode_seq(const SeqLinear *list, int n, void *workspace, const DeviceGlobals &g,
                               cudaStream_t st);
+// Prefill GEMM.  `expanded` (or null): a workspace of gemm_expanded_bytes()
+// for the weights expanded to int8, used on uniform rows from
+// kGemmExpandMinT tokens (the weights are expanded once per call and both
+// MMA operands stream in by TMA, instead of every 128-token tile decoding
+// them again).
+constexpr int64_t kGemmExpandMinT = 256;
+// The GEMM over expanded int8 weights on pairs of SMs (gemm_pair.cu).
+cudaError_t launch_gemm_pair(const void *data, int64_t rows, int64_t cols, const int8_t *q, const float *s,
+                             int64_t T, float *y, const int8_t *expanded, const DeviceGlobals &g,
+                             cudaStream_t st);
+size_t gemm_expanded_bytes(int64_t rows, int64_t cols);
 cudaError_t launch_gemm(const void *data, int64_t rows, int64_t cols, bool uniform,
                         const int8_t *q, const float *s, int64_t T, float *y, int32_t *acc,
-                        const DeviceGlobals &g, cudaStream_t st);
+                        const DeviceGlobals &g, cudaStream_t st, int8_t *expanded = nullptr);
 
 }  // namespace bitnet

@@ -32,6 +32,12 @@
 // bit, waits (bounded) for its own copies and MMAs in flight, frees tensor
 // memory and returns.  Launched with programmatic dependent launch: set-up
 // overlaps the previous kernel; q and s are read only after it has finished.
+//
+// With a caller's workspace, from kGemmExpandMinT tokens on uniform rows, the
+// weights are instead expanded to int8 once per call (expand_weights_kernel
+// below) and the pair kernel of gemm_pair.cu multiplies with both operands
+// loaded by TMA: here every 128-token tile decodes its weights again, which
+// at 2048 tokens is sixteen decodes of each weight.
 #include <cudaTypedefs.h>
 
 #include "common.cuh"
@@ -65,6 +71,7 @@ struct Cfg {
     static constexpr int kOffScale = kOffOut + kOutBytes;
     static constexpr int kOffBar = kOffScale + kScaleBytes;
     static constexpr size_t kSmem = 1024 + (size_t)kOffBar + kBarBytes;
+    static_assert(kSmem <= 227 * 1024, "shared memory");
     static_assert(kStageBytes % 1024 == 0, "stage must keep 1024-byte alignment");
     static_assert(kTmemCols >= 32 && kTmemCols <= 512 && (kTmemCols & (kTmemCols - 1)) == 0, "tmem cols");
 };
@@ -413,6 +420,48 @@ gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ C
     if (warp == 1) ptx::tmem_dealloc(tmem, C::kTmemCols);
 }
 
+// Expands the repacked code tiles to int8 t = c - 1, row-major [ntr * 16]
+// [cols].  One warp per 512-byte tile (16 rows x 128 weights): lane 4g+t
+// holds bytes 4t.. of row g (x) and of row g+8 (y) and bytes 16+4t.. of the
+// same rows (z, w); byte b of a row's block holds weights b + 32 grp at shift
+// 6 - 2 grp.  The warp stages the tile in shared memory and each lane then
+// writes whole 16-byte pieces of output rows, eight lanes to a 128-byte row:
+// piece c of row r is group c / 2, words (c & 1) * 4 .. + 3 of the row, i.e.
+// the x (or z; y, w for rows 8..15) words of lanes 4g .. 4g+3 decoded at that
+// group's shift.  The code words are read before griddepcontrol.wait (no
+// kernel writes weights); the output, which the previous kernel may still be
+// reading, is written after it.
+constexpr int kExpandWarps = 8;
+__global__ void __launch_bounds__(32 * kExpandWarps) expand_weights_kernel(const uint4 *tiles, int8_t *out,
+                                                                           int64_t ntiles, int nb, int64_t cols) {
+    __shared__ uint4 stage[kExpandWarps][32];
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t tj = (int64_t)blockIdx.x * kExpandWarps + warp;  // tile tr * nb + j
+    const bool has = tj < ntiles;
+    const uint4 v = has ? __ldcs(tiles + tj * 32 + lane) : make_uint4(0, 0, 0, 0);
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (!has) return;
+    stage[warp][lane] = v;
+    __syncwarp();
+    const uint32_t *sw = reinterpret_cast<const uint32_t *>(stage[warp]);
+    const int j = (int)(tj % nb);
+    const int64_t tr = tj / nb;
+    const int c = lane & 7, grp = c >> 1;
+#pragma unroll
+    for (int i = 0; i < 4; i++) {
+        const int r = 4 * i + (lane >> 3);           // output row of the tile
+        const int g = r & 7;
+        const int f = (r >> 3) + 2 * (c & 1);        // word of the lane's 16 bytes: x 0, y 1, z 2, w 3
+        uint4 o;
+        o.x = decode_group(sw[(4 * g + 0) * 4 + f], grp);
+        o.y = decode_group(sw[(4 * g + 1) * 4 + f], grp);
+        o.z = decode_group(sw[(4 * g + 2) * 4 + f], grp);
+        o.w = decode_group(sw[(4 * g + 3) * 4 + f], grp);
+        *reinterpret_cast<uint4 *>(out + (tr * 16 + r) * cols + 128 * j + 16 * c) = o;
+    }
+}
+
 // ---------------------------------------------------------------- host side
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -490,9 +539,14 @@ cudaError_t run(const void *data, const Layout &L, const int8_t *q, GemmArgs a, 
 
 }  // namespace
 
+size_t gemm_expanded_bytes(int64_t rows, int64_t cols) {
+    const Layout L = layout_of(rows, cols);
+    return (size_t)L.ntr * kTileRows * (size_t)L.cols;
+}
+
 cudaError_t launch_gemm(const void *data, int64_t rows, int64_t cols, bool uniform, const int8_t *q,
                         const float *s, int64_t T, float *y, int32_t *acc, const DeviceGlobals &g,
-                        cudaStream_t st) {
+                        cudaStream_t st, int8_t *expanded) {
     const Layout L = layout_of(rows, cols);
     const char *base = static_cast<const char *>(data);
     GemmArgs a;
@@ -510,6 +564,24 @@ cudaError_t launch_gemm(const void *data, int64_t rows, int64_t cols, bool unifo
     a.ntiles = 0;
     a.tma_store = 0;
     if (acc) return run<64, true, true>(data, L, q, a, st);
+    if (uniform && expanded && T >= kGemmExpandMinT) {
+        // Expand the weights once, then both operands stream in by TMA.
+        const int64_t ntiles = L.ntr * L.nb;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)((ntiles + kExpandWarps - 1) / kExpandWarps));
+        cfg.blockDim = dim3(32 * kExpandWarps);
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        cudaError_t e = cudaLaunchKernelEx(&cfg, expand_weights_kernel,
+                                           reinterpret_cast<const uint4 *>(base + L.off_tiles), expanded, ntiles,
+                                           (int)L.nb, (int64_t)L.cols);
+        if (e != cudaSuccess) return e;
+        return launch_gemm_pair(data, rows, cols, q, s, T, y, expanded, g, st);
+    }
     if (uniform) return run<256, false, false>(data, L, q, a, st);
     return run<64, true, false>(data, L, q, a, st);
 }
