@@ -910,7 +910,8 @@ def run_case(args):
     """One kernel on one shape, for profiling: `--case gemv` runs
     bitnet_w2a8_gemv (batch `--batch`), `--case linear` bitnet_w2a8_linear,
     both over `--copies` distinct weights (so the weights exceed L2); `--case
-    gemm` runs bitnet_w2a8_gemm on one weight (`--tokens`); `--case quant`
+    gemm` runs bitnet_w2a8_gemm on one weight (`--tokens`), `--case gemm_ws`
+    bitnet_w2a8_gemm_ws (weights expanded into a workspace); `--case quant`
     bitnet_quant_act on `--tokens` rows; `--case seq` one bitnet_w2a8_linear_seq
     call over `--copies` linears of the shape; `--case step` the benchmark's
     step (timed from graph replays).  `--reps` passes, plain launches (no
@@ -956,6 +957,9 @@ def run_case(args):
         calls = [lambda w=ws[(c, "w")]: b.bitnet_w2a8_gemv(w, q, s, T, y[:T * o]) for c in range(copies)]
     elif args.case == "quant":
         calls = [lambda: b.bitnet_quant_act(x, T, k, q, s)]
+    elif args.case == "gemm_ws":
+        wsp = torch.empty(b.bitnet_w2a8_gemm_workspace_bytes(o, k), dtype=torch.uint8, device=dev)
+        calls = [lambda: b.bitnet_w2a8_gemm_ws(ws[(0, "w")], q, s, T, y[:T * o], wsp)]
     else:
         calls = [lambda: b.bitnet_w2a8_gemm(ws[(0, "w")], q, s, T, y[:T * o])]
     if args.case == "step":
@@ -998,7 +1002,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--case", choices=["gemv", "linear", "gemm", "quant", "seq", "step"],
+    ap.add_argument("--case", choices=["gemv", "linear", "gemm", "gemm_ws", "quant", "seq", "step"],
                     help="profile one kernel on one shape (step: the benchmark's sequence call)")
     ap.add_argument("--rows", type=int, default=13824)
     ap.add_argument("--cols", type=int, default=2560)
