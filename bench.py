@@ -575,8 +575,9 @@ def run_llama8b(b, torch, dev, T, peaks):
 def prefill_shapes(b, torch, dev, T, peaks, cases, tokens):
     """Per shape: bitnet_w2a8_gemm (weights decoded in the kernel, per
     128-token tile), bitnet_w2a8_gemm_ws (weights expanded to int8 once per
-    call, then the pair-of-SMs GEMM), the quantiser, and the quantiser
-    followed by each GEMM (the prefill linear, x fp32 -> y)."""
+    call, then the pair-of-SMs GEMM), the quantiser, the quantiser followed
+    by bitnet_w2a8_gemm (linear_us), and bitnet_w2a8_linear_ws (linear_ws_us:
+    one kernel quantises x and expands the weights, then the pair GEMM)."""
     out = {}
     for name, o, k, w in cases:
         x = torch.randn(tokens * k, dtype=torch.float32, device=dev)
@@ -588,8 +589,7 @@ def prefill_shapes(b, torch, dev, T, peaks, cases, tokens):
         g_m = T.capture(lambda: b.bitnet_w2a8_gemm(w, q, s, tokens, y))
         g_w = T.capture(lambda: b.bitnet_w2a8_gemm_ws(w, q, s, tokens, y, ws))
         g_b = T.capture(lambda: (b.bitnet_quant_act(x, tokens, k, q, s), b.bitnet_w2a8_gemm(w, q, s, tokens, y)))
-        g_bw = T.capture(lambda: (b.bitnet_quant_act(x, tokens, k, q, s),
-                                  b.bitnet_w2a8_gemm_ws(w, q, s, tokens, y, ws)))
+        g_bw = T.capture(lambda: b.bitnet_w2a8_linear_ws(w, x, tokens, y, q, s, ws))
         mq, mm, mw, mb, mbw = T.ms(g_q, 10), T.ms(g_m, 10), T.ms(g_w, 10), T.ms(g_b, 10), T.ms(g_bw, 10)
         ops = 2.0 * tokens * o * k
         tops = ops / (mm * 1e-3) / 1e12

@@ -254,6 +254,23 @@ bitnet_status bitnet_w2a8_gemv(const bitnet_weight *w, const int8_t *q_dev, cons
 bitnet_status bitnet_w2a8_linear(const bitnet_weight *w, const float *x_dev, int64_t B, float *y_dev,
                                  int8_t *q_out_dev, float *s_out_dev, bitnet_stream_t stream);
 
+/* Linear layer for any token count T >= 1 (prefill): quantises fp32 x
+ * [T][K] exactly as bitnet_quant_act does into q_out_dev / s_out_dev
+ * (required), then computes y [T][rows] as bitnet_w2a8_gemm (T > 64) or
+ * bitnet_w2a8_linear (T <= 64) does, bit for bit.  With a workspace of
+ * bitnet_w2a8_gemm_workspace_bytes(rows, cols) (or NULL), on uniform rows
+ * from 256 tokens and K <= 32768, ONE kernel quantises x and expands the
+ * weights into the workspace side by side, then the GEMM of
+ * bitnet_w2a8_gemm_ws runs; otherwise the quantiser, then the GEMM.
+ * x_dev, y_dev, q_out_dev: 16-byte aligned; s_out_dev 4; workspace_dev 256
+ * (caller owned, stream ordered as for bitnet_w2a8_gemm_ws).
+ * Errors: NULL, SHAPE, ALIGN, VALUE, BUFSIZE (workspace), UNSUPPORTED (T > 64
+ * on a device that is not sm_100), CUDA; bounded device waits latch
+ * BITNET_ERR_TIMEOUT. */
+bitnet_status bitnet_w2a8_linear_ws(const bitnet_weight *w, const float *x_dev, int64_t T, float *y_dev,
+                                    int8_t *q_out_dev, float *s_out_dev, void *workspace_dev, size_t workspace_bytes,
+                                    bitnet_stream_t stream);
+
 /* A sequence of batch-1 decode linears in ONE persistent kernel.  Each entry
  * computes exactly what bitnet_w2a8_linear computes with B = 1 on uniform rows
  * (same q, s, int32 sums and fp32 epilogue, bit for bit): per-token absmax

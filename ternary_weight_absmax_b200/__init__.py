@@ -87,6 +87,7 @@ def _load() -> ctypes.CDLL:
         "bitnet_w2a8_gemm": ([W, vp, vp, i64, vp, vp], st),
         "bitnet_w2a8_gemm_workspace_bytes": ([i64, i64], sz),
         "bitnet_w2a8_gemm_ws": ([W, vp, vp, i64, vp, vp, sz, vp], st),
+        "bitnet_w2a8_linear_ws": ([W, vp, i64, vp, vp, vp, vp, sz, vp], st),
         "bitnet_w2a8_linear": ([W, vp, i64, vp, vp, vp, vp], st),
         "bitnet_w2a8_linear_acc": ([W, vp, i64, vp, vp, vp, vp, vp], st),
         "bitnet_w2a8_gemv_acc": ([W, vp, vp, i64, vp, vp, vp], st),
@@ -286,6 +287,18 @@ def bitnet_w2a8_gemm_ws(w: Weight, q, s, T: int, y, workspace, stream=None):
                                     _dptr(y, "float32", T * w.rows, "y"), ws,
                                     workspace.numel() if workspace is not None else 0, _stream(stream)),
            "bitnet_w2a8_gemm_ws")
+
+
+def bitnet_w2a8_linear_ws(w: Weight, x, T: int, y, q_out, s_out, workspace=None, stream=None):
+    """Linear layer at any T: fp32 x [T*K] -> y [T*rows], q_out / s_out written;
+    workspace: uint8 CUDA tensor of bitnet_w2a8_gemm_workspace_bytes(rows, cols) or None."""
+    n = bitnet_w2a8_gemm_workspace_bytes(w.rows, w.cols)
+    ws = _dptr(workspace, "uint8", n, "workspace") if workspace is not None else None
+    _check(_lib.bitnet_w2a8_linear_ws(w.ref(), _dptr(x, "float32", T * w.cols, "x"), T,
+                                      _dptr(y, "float32", T * w.rows, "y"), _dptr(q_out, "int8", T * w.cols, "q_out"),
+                                      _dptr(s_out, "float32", T, "s_out"), ws,
+                                      workspace.numel() if workspace is not None else 0, _stream(stream)),
+           "bitnet_w2a8_linear_ws")
 
 
 def bitnet_w2a8_linear(w: Weight, x, B: int, y, q_out=None, s_out=None, stream=None):

@@ -354,6 +354,48 @@ bitnet_status bitnet_w2a8_linear_acc(const bitnet_weight *w, const float *x_dev,
     return linear_impl(w, x_dev, B, y_dev, q_out_dev, s_out_dev, acc_dev, stream);
 }
 
+bitnet_status bitnet_w2a8_linear_ws(const bitnet_weight *w, const float *x_dev, int64_t T, float *y_dev,
+                                    int8_t *q_out_dev, float *s_out_dev, void *workspace_dev, size_t workspace_bytes,
+                                    bitnet_stream_t stream) {
+    t_detail[0] = 0;
+    bitnet_status s = check_weight(w);
+    if (s != BITNET_OK) return s;
+    if (T < 1 || T >= kMaxT) return fail(BITNET_ERR_SHAPE, "T=%lld invalid", (long long)T);
+    if (!x_dev || !y_dev || !q_out_dev || !s_out_dev) return fail(BITNET_ERR_NULL, "NULL pointer");
+    if (!aligned(x_dev, 16) || !aligned(y_dev, 16) || !aligned(q_out_dev, 16) || !aligned(s_out_dev, 4))
+        return fail(BITNET_ERR_ALIGN, "x, y and q_out need 16-byte, s_out 4-byte alignment");
+    if (workspace_dev) {
+        if (!aligned(workspace_dev, 256)) return fail(BITNET_ERR_ALIGN, "workspace needs 256-byte alignment");
+        if (workspace_bytes < gemm_expanded_bytes(w->rows, w->cols))
+            return fail(BITNET_ERR_BUFSIZE, "workspace %zu < %zu bytes", workspace_bytes,
+                        gemm_expanded_bytes(w->rows, w->cols));
+    }
+    if (T <= 64) return linear_impl(w, x_dev, T, y_dev, q_out_dev, s_out_dev, nullptr, stream);
+    int dev = 0, major = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    if (e != cudaSuccess) return cuda_fail(e, "device query");
+    if (major != 10) return fail(BITNET_ERR_UNSUPPORTED, "GEMM needs an sm_100 device (found sm_%d)", major * 10);
+    DeviceGlobals g;
+    e = device_globals(&g);
+    if (e != cudaSuccess) return cuda_fail(e, "device globals");
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const bool uniform = (w->flags & BITNET_WEIGHT_UNIFORM_ROWS) != 0;
+    int8_t *ws = static_cast<int8_t *>(workspace_dev);
+    if (uniform && ws && T >= kGemmExpandMinT && prefill_prep_supported(w->cols)) {
+        // One kernel quantises x and expands the weights side by side, then
+        // the pair-of-SMs GEMM.
+        e = launch_prefill_prep(x_dev, T, w->cols, q_out_dev, s_out_dev, w->data, w->rows, ws, st);
+        if (e == cudaSuccess)
+            e = launch_gemm_pair(w->data, w->rows, w->cols, q_out_dev, s_out_dev, T, y_dev, ws, g, st);
+    } else {
+        e = launch_quant_act(x_dev, T, w->cols, q_out_dev, s_out_dev, nullptr, st);
+        if (e == cudaSuccess)
+            e = launch_gemm(w->data, w->rows, w->cols, uniform, q_out_dev, s_out_dev, T, y_dev, nullptr, g, st, ws);
+    }
+    return e == cudaSuccess ? BITNET_OK : cuda_fail(e, "linear_ws launch");
+}
+
 bitnet_status bitnet_w2a8_gemv(const bitnet_weight *w, const int8_t *q_dev, const float *s_dev, int64_t B,
                                float *y_dev, bitnet_stream_t stream) {
     return gemv_impl(w, q_dev, s_dev, B, y_dev, nullptr, stream);

@@ -67,6 +67,11 @@ cudaError_t device_globals(DeviceGlobals *out);
 int num_sms();
 
 // Launchers (return the launch error, if any).
+// The prefill linear's pre-pass: quantise x (T rows) and expand the weights
+// into `expanded` in one kernel (quant_act.cu); K up to 32768.
+bool prefill_prep_supported(int64_t K);
+cudaError_t launch_prefill_prep(const float *x, int64_t T, int64_t K, int8_t *q, float *s, const void *data,
+                                int64_t rows, int8_t *expanded, cudaStream_t st);
 cudaError_t launch_quant_act(const float *x, int64_t T, int64_t K, int8_t *q, float *s,
                              int32_t *blocksum, cudaStream_t st);
 cudaError_t launch_repack(const uint8_t *codes, const float *scales, int64_t rows, int64_t cols,

@@ -41,6 +41,7 @@
 #include <cudaTypedefs.h>
 
 #include "common.cuh"
+#include "expand.cuh"
 #include "tcgen05.cuh"
 
 namespace bitnet {
@@ -93,11 +94,6 @@ struct GemmArgs {
 
 __device__ __forceinline__ uint32_t sw128_offset(int n, int k) {
     return (uint32_t)((n >> 3) * 1024 + (n & 7) * 128 + ((((k >> 4) ^ (n & 7)) << 4) | (k & 15)));
-}
-
-__device__ __forceinline__ uint32_t decode_group(uint32_t w, int grp) {
-    const uint32_t c = (w >> (6 - 2 * grp)) & 0x03030303u;
-    return (c + 0x7F7F7F7Fu) ^ 0x80808080u;
 }
 
 // Bounded wait by lane 0 only, result broadcast to the warp, so every lane of a
@@ -284,10 +280,10 @@ gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ C
 #pragma unroll
                     for (int grp = 0; grp < 4; grp++) {
                         const int k0 = 32 * grp + 4 * t, k1 = k0 + 16;
-                        *reinterpret_cast<uint32_t *>(bs + sw128_offset(na, k0)) = decode_group(c.x, grp);
-                        *reinterpret_cast<uint32_t *>(bs + sw128_offset(nbr, k0)) = decode_group(c.y, grp);
-                        *reinterpret_cast<uint32_t *>(bs + sw128_offset(na, k1)) = decode_group(c.z, grp);
-                        *reinterpret_cast<uint32_t *>(bs + sw128_offset(nbr, k1)) = decode_group(c.w, grp);
+                        *reinterpret_cast<uint32_t *>(bs + sw128_offset(na, k0)) = expand_group(c.x, grp);
+                        *reinterpret_cast<uint32_t *>(bs + sw128_offset(nbr, k0)) = expand_group(c.y, grp);
+                        *reinterpret_cast<uint32_t *>(bs + sw128_offset(na, k1)) = expand_group(c.z, grp);
+                        *reinterpret_cast<uint32_t *>(bs + sw128_offset(nbr, k1)) = expand_group(c.w, grp);
                     }
                 }
                 ptx::fence_proxy_async_smem();
@@ -421,16 +417,9 @@ gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ C
 }
 
 // Expands the repacked code tiles to int8 t = c - 1, row-major [ntr * 16]
-// [cols].  One warp per 512-byte tile (16 rows x 128 weights): lane 4g+t
-// holds bytes 4t.. of row g (x) and of row g+8 (y) and bytes 16+4t.. of the
-// same rows (z, w); byte b of a row's block holds weights b + 32 grp at shift
-// 6 - 2 grp.  The warp stages the tile in shared memory and each lane then
-// writes whole 16-byte pieces of output rows, eight lanes to a 128-byte row:
-// piece c of row r is group c / 2, words (c & 1) * 4 .. + 3 of the row, i.e.
-// the x (or z; y, w for rows 8..15) words of lanes 4g .. 4g+3 decoded at that
-// group's shift.  The code words are read before griddepcontrol.wait (no
-// kernel writes weights); the output, which the previous kernel may still be
-// reading, is written after it.
+// [cols], one warp per tile (expand.cuh).  The code words are read before
+// griddepcontrol.wait (no kernel writes weights); the output, which the
+// previous kernel may still be reading, is written after it.
 constexpr int kExpandWarps = 8;
 __global__ void __launch_bounds__(32 * kExpandWarps) expand_weights_kernel(const uint4 *tiles, int8_t *out,
                                                                            int64_t ntiles, int nb, int64_t cols) {
@@ -441,25 +430,7 @@ __global__ void __launch_bounds__(32 * kExpandWarps) expand_weights_kernel(const
     const bool has = tj < ntiles;
     const uint4 v = has ? __ldcs(tiles + tj * 32 + lane) : make_uint4(0, 0, 0, 0);
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    if (!has) return;
-    stage[warp][lane] = v;
-    __syncwarp();
-    const uint32_t *sw = reinterpret_cast<const uint32_t *>(stage[warp]);
-    const int j = (int)(tj % nb);
-    const int64_t tr = tj / nb;
-    const int c = lane & 7, grp = c >> 1;
-#pragma unroll
-    for (int i = 0; i < 4; i++) {
-        const int r = 4 * i + (lane >> 3);           // output row of the tile
-        const int g = r & 7;
-        const int f = (r >> 3) + 2 * (c & 1);        // word of the lane's 16 bytes: x 0, y 1, z 2, w 3
-        uint4 o;
-        o.x = decode_group(sw[(4 * g + 0) * 4 + f], grp);
-        o.y = decode_group(sw[(4 * g + 1) * 4 + f], grp);
-        o.z = decode_group(sw[(4 * g + 2) * 4 + f], grp);
-        o.w = decode_group(sw[(4 * g + 3) * 4 + f], grp);
-        *reinterpret_cast<uint4 *>(out + (tr * 16 + r) * cols + 128 * j + 16 * c) = o;
-    }
+    if (has) expand_tile(v, stage[warp], out, tj, nb, cols);
 }
 
 // ---------------------------------------------------------------- host side

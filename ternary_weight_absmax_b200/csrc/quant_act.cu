@@ -19,6 +19,7 @@
 #include <atomic>
 
 #include "common.cuh"
+#include "expand.cuh"
 
 namespace bitnet {
 namespace {
@@ -33,20 +34,14 @@ __device__ __forceinline__ int quant_one(float x, float s) {
     return v;
 }
 
+// Row `row` of x by the whole CTA (red: kMaxThreads / 32 floats of shared memory).
 template <int NPER, bool kBlockSum>
-__global__ void __launch_bounds__(kMaxThreads)
-quant_act_kernel(const float4 *__restrict__ x, int64_t K, int8_t *__restrict__ q,
-                 float *__restrict__ s, int32_t *__restrict__ blocksum) {
-    // x may be produced by the kernel just before on the stream: wait for it
-    // (a no-op without programmatic dependent launch), then let the next
-    // kernel launch so it can prefetch its weights while this one runs.
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    const int64_t row = blockIdx.x;
+__device__ __forceinline__ void quant_row(const float4 *__restrict__ x, int64_t K, int8_t *__restrict__ q,
+                                          float *__restrict__ s, int32_t *__restrict__ blocksum, int64_t row,
+                                          float *red) {
     const int n4 = (int)(K / 4);
     const float4 *xr = x + row * n4;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nt = blockDim.x;
-    __shared__ float red[kMaxThreads / 32];
 
     float4 v[NPER];
     float m = 0.0f;
@@ -87,6 +82,46 @@ quant_act_kernel(const float4 *__restrict__ x, int64_t K, int8_t *__restrict__ q
             if (lane == 0 && blk * 32 < n4) blocksum[row * (K / 128) + blk] = sum;
         }
     }
+}
+
+template <int NPER, bool kBlockSum>
+__global__ void __launch_bounds__(kMaxThreads)
+quant_act_kernel(const float4 *__restrict__ x, int64_t K, int8_t *__restrict__ q,
+                 float *__restrict__ s, int32_t *__restrict__ blocksum) {
+    // x may be produced by the kernel just before on the stream: wait for it
+    // (a no-op without programmatic dependent launch), then let the next
+    // kernel launch so it can prefetch its weights while this one runs.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    __shared__ float red[kMaxThreads / 32];
+    quant_row<NPER, kBlockSum>(x, K, q, s, blocksum, blockIdx.x, red);
+}
+
+// The prefill linear's pre-pass: CTAs 0 .. T-1 quantise the token rows (as
+// quant_act_kernel), the others expand the weights to int8 for the GEMM, one
+// warp per 512-byte code tile (expand.cuh), so the two run side by side.
+// Both write only after griddepcontrol.wait (x may come from the previous
+// kernel, which may also still read the workspace); the code words are read
+// before it.
+template <int NPER>
+__global__ void __launch_bounds__(kMaxThreads)
+prefill_prep_kernel(const float4 *__restrict__ x, int64_t K, int8_t *__restrict__ q, float *__restrict__ s,
+                    int64_t T, const uint4 *__restrict__ tiles, int8_t *__restrict__ wout, int64_t ntiles,
+                    int nb) {
+    __shared__ float red[kMaxThreads / 32];
+    __shared__ uint4 stage[kMaxThreads / 32][32];
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    if ((int64_t)blockIdx.x < T) {
+        asm volatile("griddepcontrol.wait;" ::: "memory");
+        quant_row<NPER, false>(x, K, q, s, nullptr, blockIdx.x, red);
+        return;
+    }
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t tj = ((int64_t)blockIdx.x - T) * (blockDim.x >> 5) + warp;  // tile tr * nb + j
+    const bool has = tj < ntiles;
+    const uint4 v = has ? __ldcs(tiles + tj * 32 + lane) : make_uint4(0, 0, 0, 0);
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (has) expand_tile(v, stage[warp], wout, tj, nb, K);
 }
 
 // Rows longer than 16 float4 per thread of 512 threads (K > 32768): two
@@ -144,6 +179,42 @@ cudaError_t launch_one(const cudaLaunchConfig_t &cfg, const float4 *x4, int64_t 
 }
 
 }  // namespace
+
+bool prefill_prep_supported(int64_t K) { return K / 4 <= 16 * (int64_t)kMaxThreads; }
+
+cudaError_t launch_prefill_prep(const float *x, int64_t T, int64_t K, int8_t *q, float *s, const void *data,
+                                int64_t rows, int8_t *expanded, cudaStream_t st) {
+    if (T == 0) return cudaSuccess;
+    const int64_t n4 = K / 4;
+    int nper = 1;
+    while (nper < 16 && n4 > (int64_t)nper * kMaxThreads) nper *= 2;
+    if (n4 > (int64_t)nper * kMaxThreads) return cudaErrorInvalidValue;  // rows of K > 32768: not taken
+    int64_t threads = (n4 + nper - 1) / nper;
+    threads = (threads + 31) / 32 * 32;
+    const Layout L = layout_of(rows, K);
+    const int64_t ntiles = L.ntr * L.nb;
+    const int64_t warps = threads / 32;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(T + (ntiles + warps - 1) / warps));
+    cfg.blockDim = dim3((unsigned)threads);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const float4 *x4 = reinterpret_cast<const float4 *>(x);
+    const uint4 *tiles = reinterpret_cast<const uint4 *>(static_cast<const char *>(data) + L.off_tiles);
+    const int nb = (int)L.nb;
+    switch (nper) {
+        case 1: return cudaLaunchKernelEx(&cfg, prefill_prep_kernel<1>, x4, K, q, s, T, tiles, expanded, ntiles, nb);
+        case 2: return cudaLaunchKernelEx(&cfg, prefill_prep_kernel<2>, x4, K, q, s, T, tiles, expanded, ntiles, nb);
+        case 4: return cudaLaunchKernelEx(&cfg, prefill_prep_kernel<4>, x4, K, q, s, T, tiles, expanded, ntiles, nb);
+        case 8: return cudaLaunchKernelEx(&cfg, prefill_prep_kernel<8>, x4, K, q, s, T, tiles, expanded, ntiles, nb);
+        default:
+            return cudaLaunchKernelEx(&cfg, prefill_prep_kernel<16>, x4, K, q, s, T, tiles, expanded, ntiles, nb);
+    }
+}
 
 cudaError_t launch_quant_act(const float *x, int64_t T, int64_t K, int8_t *q, float *s,
                              int32_t *blocksum, cudaStream_t st) {

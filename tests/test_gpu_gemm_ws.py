@@ -5,6 +5,9 @@ s = 1: y is the sum itself) and the same y, bit for bit, as
 bitnet_w2a8_gemm on every shape, including rows that end inside a 256-row
 tile and token counts that end inside a 128-token tile; below 256 tokens,
 on block-scale weights and without a workspace it is bitnet_w2a8_gemm.
+bitnet_w2a8_linear_ws (fp32 x in; from 256 tokens with a workspace one
+kernel quantises x and expands the weights) must give the q, s and y of the
+quantiser followed by bitnet_w2a8_gemm, bit for bit.
 The product is the integer add / subtract / skip of the ternary weights
 ("BitRun v0.2 实测：1-bit LLM 终端驾驶舱与毫瓦级功耗遥测", section
 "三值权重与 1.58-bit 的由来")."""
@@ -175,3 +178,57 @@ def test_gemm_ws_wait_timeout_is_reported_and_recoverable():
     assert b.bitnet_get_device_error() == b.BITNET_OK
     rq, rs, _ = oracle.quant_act(x)
     assert_close(to_np(y).reshape(T, rows), oracle.linear(oracle.pack_i2s(t), sc, K, rq, rs), "after timeout")
+
+
+@pytest.mark.parametrize("rows,K,T,mode,with_ws", [
+    (256, 512, 64, "tensor", True), (300, 640, 100, "tensor", True), (1000, 1280, 300, "tensor", True),
+    (13824, 2560, 2048, "tensor", True), (2560, 6912, 512, "tensor", True), (2576, 2560, 257, "tensor", True),
+    (300, 640, 300, "tensor", False), (256, 512, 512, "block", True),
+])
+def test_linear_ws_matches_quantiser_then_gemm(rows, K, T, mode, with_ws):
+    # bitnet_w2a8_linear_ws (from 256 tokens with a workspace: one kernel that
+    # quantises x and expands the weights, then the pair GEMM) against the
+    # quantiser followed by bitnet_w2a8_gemm (bitnet_w2a8_linear up to 64
+    # tokens): q, s and y bit for bit.
+    b = lib()
+    tt = torch()
+    t = syn.ternary_uniform(rows * 5 + T, rows, K)
+    sc = syn.positive_scales(rows + 3, rows, K // QK, per_tensor=(mode == "tensor"))
+    x = cuda(syn.activations(K + T, T, K, outliers=True).reshape(-1))
+    w, _ = device_weight(t, sc)
+    q0 = tt.empty(T * K, dtype=tt.int8, device="cuda")
+    s0 = tt.empty(T, dtype=tt.float32, device="cuda")
+    y0 = tt.empty(T * rows, dtype=tt.float32, device="cuda")
+    if T <= 64:
+        b.bitnet_w2a8_linear(w, x, T, y0, q0, s0)
+    else:
+        b.bitnet_quant_act(x, T, K, q0, s0)
+        b.bitnet_w2a8_gemm(w, q0, s0, T, y0)
+    q1 = tt.full((T * K,), 99, dtype=tt.int8, device="cuda")
+    s1 = tt.full((T,), -1.0, dtype=tt.float32, device="cuda")
+    y1 = tt.full((T * rows,), float("nan"), dtype=tt.float32, device="cuda")
+    b.bitnet_w2a8_linear_ws(w, x, T, y1, q1, s1, _workspace(rows, K) if with_ws else None)
+    assert b.bitnet_get_device_error() == b.BITNET_OK
+    assert tt.equal(q0, q1) and tt.equal(s0, s1), "q or s differ"
+    assert np.array_equal(to_np(y0).view(np.uint32), to_np(y1).view(np.uint32)), f"{rows}x{K} T={T} {mode}"
+
+
+def test_linear_ws_checks_its_arguments():
+    b = lib()
+    tt = torch()
+    rows, K, T = 256, 512, 300
+    t = syn.ternary_uniform(21, rows, K)
+    w, _ = device_weight(t, syn.positive_scales(22, rows, K // QK, per_tensor=True))
+    x = tt.zeros(T * K, dtype=tt.float32, device="cuda")
+    q = tt.empty(T * K, dtype=tt.int8, device="cuda")
+    s = tt.empty(T, dtype=tt.float32, device="cuda")
+    y = tt.empty(T * rows, dtype=tt.float32, device="cuda")
+    need = b.bitnet_w2a8_gemm_workspace_bytes(rows, K)
+    ws = tt.zeros(need, dtype=tt.uint8, device="cuda")
+    raw = b.library().bitnet_w2a8_linear_ws
+    p = lambda a: ctypes.c_void_p(a.data_ptr())
+    assert raw(w.ref(), p(x), T, p(y), None, p(s), p(ws), need, None) == b.BITNET_ERR_NULL
+    assert raw(w.ref(), p(x), T, p(y), p(q), p(s), p(ws), need - 1, None) == b.BITNET_ERR_BUFSIZE
+    assert raw(w.ref(), p(x), 0, p(y), p(q), p(s), p(ws), need, None) == b.BITNET_ERR_SHAPE
+    assert raw(w.ref(), p(x), T, p(y), p(q), p(s), p(ws), need, None) == b.BITNET_OK
+    assert b.bitnet_get_device_error() == b.BITNET_OK
