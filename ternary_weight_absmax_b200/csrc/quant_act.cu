@@ -178,6 +178,12 @@ cudaError_t launch_one(const cudaLaunchConfig_t &cfg, const float4 *x4, int64_t 
     return cudaLaunchKernelEx(&cfg, quant_act_kernel<NPER, false>, x4, K, q, s, (int32_t *)nullptr);
 }
 
+template <int NPER>
+cudaError_t launch_prep(const cudaLaunchConfig_t &cfg, const float4 *x4, int64_t K, int8_t *q, float *s, int64_t T,
+                        const uint4 *tiles, int8_t *wout, int64_t ntiles, int nb) {
+    return cudaLaunchKernelEx(&cfg, prefill_prep_kernel<NPER>, x4, K, q, s, T, tiles, wout, ntiles, nb);
+}
+
 }  // namespace
 
 bool prefill_prep_supported(int64_t K) { return K / 4 <= 16 * (int64_t)kMaxThreads; }
@@ -207,12 +213,11 @@ cudaError_t launch_prefill_prep(const float *x, int64_t T, int64_t K, int8_t *q,
     const uint4 *tiles = reinterpret_cast<const uint4 *>(static_cast<const char *>(data) + L.off_tiles);
     const int nb = (int)L.nb;
     switch (nper) {
-        case 1: return cudaLaunchKernelEx(&cfg, prefill_prep_kernel<1>, x4, K, q, s, T, tiles, expanded, ntiles, nb);
-        case 2: return cudaLaunchKernelEx(&cfg, prefill_prep_kernel<2>, x4, K, q, s, T, tiles, expanded, ntiles, nb);
-        case 4: return cudaLaunchKernelEx(&cfg, prefill_prep_kernel<4>, x4, K, q, s, T, tiles, expanded, ntiles, nb);
-        case 8: return cudaLaunchKernelEx(&cfg, prefill_prep_kernel<8>, x4, K, q, s, T, tiles, expanded, ntiles, nb);
-        default:
-            return cudaLaunchKernelEx(&cfg, prefill_prep_kernel<16>, x4, K, q, s, T, tiles, expanded, ntiles, nb);
+        case 1: return launch_prep<1>(cfg, x4, K, q, s, T, tiles, expanded, ntiles, nb);
+        case 2: return launch_prep<2>(cfg, x4, K, q, s, T, tiles, expanded, ntiles, nb);
+        case 4: return launch_prep<4>(cfg, x4, K, q, s, T, tiles, expanded, ntiles, nb);
+        case 8: return launch_prep<8>(cfg, x4, K, q, s, T, tiles, expanded, ntiles, nb);
+        default: return launch_prep<16>(cfg, x4, K, q, s, T, tiles, expanded, ntiles, nb);
     }
 }
 
