@@ -201,10 +201,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_seq_kernel(const __grid_co
     const int nseg = seg_wcnt[kSeqMaxLinears / 32];
 
     // This warp's items of segment L: [i0, i1) of the segment's cnt * nb.
+    // Warp b's share of a segment's items starts at share_of(b): an even
+    // split rounded down to a multiple of four, so that with tiles of a
+    // multiple of four items the four-item step of the product loop never
+    // straddles a tile.
+    auto share_of = [](int b, int64_t items) -> int64_t {
+        return b >= kWarps ? items : (((int64_t)b * items / kWarps) & ~(int64_t)3);
+    };
     auto run_of = [&](int L, int &i0, int &i1) {
         const int64_t items = (int64_t)seg_cnt[L] * a.lin[L].nb;
-        i0 = (int)((int64_t)warp * items / kWarps);
-        i1 = (int)((int64_t)(warp + 1) * items / kWarps);
+        i0 = (int)share_of(warp, items);
+        i1 = (int)share_of(warp + 1, items);
     };
 
     // ---- issue cursor (lane 0): the next chunk of this warp's item stream.
@@ -271,7 +278,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_seq_kernel(const __grid_co
             }
         } else if (tid < kWarps * kTileRows) {
             const int b = tid / kTileRows;
-            const int64_t pos = (int64_t)b * items / kWarps;
+            const int64_t pos = share_of(b, items);
             if (b >= 1 && pos % nb != 0) {
                 eidx = tid;
                 erow = (int)((rlo + pos / nb) * kTileRows + tid % kTileRows);
@@ -420,13 +427,19 @@ __global__ void __launch_bounds__(kThreads, 1) decode_seq_kernel(const __grid_co
                 const int nt = min(kChunk, i1 - i);
                 const uint4 *wv = reinterpret_cast<const uint4 *>(ring + slot * (kChunk * kTile)) + lane;
                 for (int e = 0; e < nt;) {
-                    if (e + 4 <= nt && j + 4 < nb) {
-                        // Four items inside the current row tile: no tile change.
+                    if (e + 4 <= nt && j + 4 <= nb) {
+                        // Four items of the current row tile.
 #pragma unroll
                         for (int u = 0; u < 4; u++) item(wv[(e + u) * 32], qp + u * 8);
                         qp += 32;
                         j += 4;
                         e += 4;
+                        if (j == nb) {
+                            flush();
+                            r++;
+                            j = 0;
+                            qp = qrow;
+                        }
                     } else {
                         item(wv[e * 32], qp);
                         qp += 8;
