@@ -146,6 +146,32 @@ def test_device_calls_validate_before_touching_the_gpu(b):
     assert lib.bitnet_repack_device(16, 16, 16, 128, ctypes.byref(w2), None) == b.BITNET_ERR_ALIGN
 
 
+def test_workspace_calls_validate_before_touching_the_gpu(b):
+    # bitnet_w2a8_gemm_ws / bitnet_w2a8_linear_ws: the int8 weights plus the
+    # hand-off area, NULL / shape / alignment / workspace size rejected on the host.
+    lib = b.library()
+    w = b.bitnet_weight()
+    w.data = 256
+    w.rows, w.cols, w.bytes = 16, 128, 1 << 20
+    w.layout_version = b.BITNET_LAYOUT_VERSION
+    w.flags = b.BITNET_WEIGHT_UNIFORM_ROWS
+    need = b.bitnet_w2a8_gemm_workspace_bytes(16, 128)
+    assert need >= 16 * 128
+    assert b.bitnet_w2a8_gemm_workspace_bytes(1000, 640) >= 1008 * 640
+    assert b.bitnet_w2a8_gemm_workspace_bytes(16, 100) == 0 and b.bitnet_w2a8_gemm_workspace_bytes(0, 128) == 0
+    wr = ctypes.byref(w)
+    assert lib.bitnet_w2a8_gemm_ws(None, 16, 16, 4, 16, 256, need, None) == b.BITNET_ERR_NULL
+    assert lib.bitnet_w2a8_gemm_ws(wr, 16, 16, -1, 16, 256, need, None) == b.BITNET_ERR_SHAPE
+    assert lib.bitnet_w2a8_gemm_ws(wr, 16, 16, 0, 16, 256, need, None) == b.BITNET_OK  # T = 0: no-op
+    assert lib.bitnet_w2a8_gemm_ws(wr, 16, 16, 4, 16, 256, need - 1, None) == b.BITNET_ERR_BUFSIZE
+    assert lib.bitnet_w2a8_gemm_ws(wr, 16, 16, 4, 16, 272, need, None) == b.BITNET_ERR_ALIGN
+    assert lib.bitnet_w2a8_linear_ws(wr, 16, 4, 16, None, 16, 256, need, None) == b.BITNET_ERR_NULL
+    assert lib.bitnet_w2a8_linear_ws(wr, 16, 0, 16, 16, 16, 256, need, None) == b.BITNET_ERR_SHAPE
+    assert lib.bitnet_w2a8_linear_ws(wr, 16, 4, 8, 16, 16, 256, need, None) == b.BITNET_ERR_ALIGN
+    assert lib.bitnet_w2a8_linear_ws(wr, 16, 4, 16, 16, 16, 256, need - 1, None) == b.BITNET_ERR_BUFSIZE
+    assert lib.bitnet_w2a8_linear_ws(wr, 16, 4, 16, 16, 16, 272, need, None) == b.BITNET_ERR_ALIGN
+
+
 def test_linear_seq_validates_before_touching_the_gpu(b):
     """bitnet_w2a8_linear_seq rejects, on the host: bad counts, waits on later
     entries, overlapping outputs, reads of another entry's output without a
