@@ -232,3 +232,34 @@ def test_linear_ws_checks_its_arguments():
     assert raw(w.ref(), p(x), 0, p(y), p(q), p(s), p(ws), need, None) == b.BITNET_ERR_SHAPE
     assert raw(w.ref(), p(x), T, p(y), p(q), p(s), p(ws), need, None) == b.BITNET_OK
     assert b.bitnet_get_device_error() == b.BITNET_OK
+
+
+@pytest.mark.parametrize("rows,K,T", [(1000, 640, 300), (13824, 2560, 2048)])
+def test_linear_ws_int32_sums_exact(rows, K, T):
+    # Integer activations whose row absmax is 127 quantise to q = x with s = 1,
+    # and unit scales make y the int32 sum itself: the fused quantise-and-
+    # expand pre-pass and the pair GEMM must reproduce the oracle's sums.
+    b = lib()
+    tt = torch()
+    seed = rows + 7 * T
+    t = syn.ternary_uniform(seed, rows, K)
+    sc = np.ones((rows, K // QK), dtype=np.float32)
+    x = syn.integer_rows(seed + 1, T, K)
+    rq, rs, _ = oracle.quant_act(x)
+    assert np.all(rs == 1.0)
+    pick = None
+    if rows * T > 10**6:
+        pick = np.unique(np.concatenate([[0, rows - 1], syn.splitmix64(seed, np.arange(48)) % np.uint64(rows)]))
+        pick = pick.astype(np.int64)
+    tp = t if pick is None else t[pick]
+    sums = oracle.block_acc(oracle.pack_i2s(tp), K, rq).astype(np.int64).sum(axis=-1)
+    w, _ = device_weight(t, sc)
+    q = tt.empty(T * K, dtype=tt.int8, device="cuda")
+    s = tt.empty(T, dtype=tt.float32, device="cuda")
+    y = tt.empty(T * rows, dtype=tt.float32, device="cuda")
+    b.bitnet_w2a8_linear_ws(w, cuda(x.reshape(-1)), T, y, q, s, _workspace(rows, K))
+    assert b.bitnet_get_device_error() == b.BITNET_OK
+    np.testing.assert_array_equal(to_np(q).reshape(T, K), rq)
+    got = to_np(y).reshape(T, rows)
+    got = got if pick is None else got[:, pick]
+    assert np.array_equal(got, sums.astype(np.float32)), f"linear_ws {rows}x{K} T={T}: int32 sums differ"
