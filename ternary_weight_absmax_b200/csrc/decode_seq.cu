@@ -218,27 +218,31 @@ __global__ void __launch_bounds__(kThreads, 1) decode_seq_kernel(const __grid_co
     const uint64_t pol = ptx::policy_evict_first();
     int ik = -1, iL = -1, ii = 0, iend = 0;  // segment, its linear, next item, end of its run
     uint32_t iq = 0;                         // chunks issued
+    const unsigned char *isrc = nullptr;     // the next chunk's first tile
     auto next_run = [&]() {
         while (++ik < nseg) {
             iL = seg_list[ik];
             run_of(iL, ii, iend);
-            if (iend > ii) return;
+            if (iend > ii) {
+                const SeqLin &l = a.lin[iL];
+                isrc = l.tiles + ((size_t)seg_lo[iL] * l.nb + ii) * kTile;
+                return;
+            }
         }
         iL = n;
     };
     uint32_t islot = 0;  // slot of the next chunk issued (iq mod kSlots)
     auto issue = [&]() {
         if (iL >= n) return;
-        const SeqLin &l = a.lin[iL];
         const int nt = min(kChunk, iend - ii);
         const uint32_t slot = islot;
         islot = islot + 1 == kSlots ? 0u : islot + 1;
         const uint32_t bar = bar0 + 8u * slot;
         ptx::mbar_arrive_expect_tx(bar, (uint32_t)(nt * kTile));
-        ptx::bulk_g2s(ptx::smem_u32(ring + slot * (kChunk * kTile)),
-                      l.tiles + ((size_t)seg_lo[iL] * l.nb + ii) * kTile, (uint32_t)(nt * kTile), bar, pol);
+        ptx::bulk_g2s(ptx::smem_u32(ring + slot * (kChunk * kTile)), isrc, (uint32_t)(nt * kTile), bar, pol);
         iq++;
         ii += nt;
+        isrc += (size_t)nt * kTile;
         if (ii >= iend) next_run();
     };
     // The first segment's x into L2 ahead of the weight copies (a prefetch
