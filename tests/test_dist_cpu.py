@@ -52,3 +52,31 @@ def test_step_bytes_accounting():
     per = sum(o * k // 4 + 4 * o + k + 4 + 4 * o for _, o, k in bench.SHAPES)
     assert g == 30 * per
     assert q == 30 * sum(5 * k + 4 for _, _, k in bench.SHAPES)
+
+
+def test_read_traffic_scales_and_checks_the_source_digest(tmp_path, monkeypatch):
+    # The roofline's traffic comes from a committed ncu record; it is scaled to
+    # the launch's algorithmic bytes and reported as null once the kernel's
+    # sources differ from those the record was taken on.
+    csrc = tmp_path / "ternary_weight_absmax_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    (tmp_path / "profiles").mkdir()
+    src = csrc / "k.cu"
+    src.write_text("// kernel, first version\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    rec = {"k": {"dram_bytes": 1000, "algorithmic_bytes": 500, "case": "a small case",
+                 "sources": ["k.cu"], "source_digest": bench.source_digest("k.cu")}}
+    import json
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(rec))
+    assert bench.read_traffic("k", 500)[0] == 1000
+    traffic, note = bench.read_traffic("k", 1500)
+    assert traffic == 3000 and "scaled" in note
+    assert bench.read_traffic("other", 500) == (None, "no ncu capture on record")
+    src.write_text("// kernel, changed\n")
+    assert bench.read_traffic("k", 500) == (None, "kernel changed since the ncu capture")
+
+
+def test_headline_bytes_per_step():
+    # codes out*K/4 + a fp32 scale per row + fp32 x + fp32 y, over the 120 linears
+    per = sum(o * k // 4 + 4 * o + 4 * k + 4 * o for _, o, k in bench.SHAPES)
+    assert bench.fused_step_bytes() == 30 * per == 528230400
