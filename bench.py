@@ -911,7 +911,8 @@ def run_case(args):
     bitnet_w2a8_gemv (batch `--batch`), `--case linear` bitnet_w2a8_linear,
     both over `--copies` distinct weights (so the weights exceed L2); `--case
     gemm` runs bitnet_w2a8_gemm on one weight (`--tokens`), `--case gemm_ws`
-    bitnet_w2a8_gemm_ws (weights expanded into a workspace); `--case quant`
+    bitnet_w2a8_gemm_ws (weights expanded into a workspace), `--case
+    linear_ws` bitnet_w2a8_linear_ws (fp32 x in); `--case quant`
     bitnet_quant_act on `--tokens` rows; `--case seq` one bitnet_w2a8_linear_seq
     call over `--copies` linears of the shape; `--case step` the benchmark's
     step (timed from graph replays).  `--reps` passes, plain launches (no
@@ -960,6 +961,9 @@ def run_case(args):
     elif args.case == "gemm_ws":
         wsp = torch.empty(b.bitnet_w2a8_gemm_workspace_bytes(o, k), dtype=torch.uint8, device=dev)
         calls = [lambda: b.bitnet_w2a8_gemm_ws(ws[(0, "w")], q, s, T, y[:T * o], wsp)]
+    elif args.case == "linear_ws":
+        wsp = torch.empty(b.bitnet_w2a8_gemm_workspace_bytes(o, k), dtype=torch.uint8, device=dev)
+        calls = [lambda: b.bitnet_w2a8_linear_ws(ws[(0, "w")], x, T, y[:T * o], q, s, wsp)]
     else:
         calls = [lambda: b.bitnet_w2a8_gemm(ws[(0, "w")], q, s, T, y[:T * o])]
     if args.case == "step":
@@ -1002,7 +1006,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--case", choices=["gemv", "linear", "gemm", "gemm_ws", "quant", "seq", "step"],
+    ap.add_argument("--case", choices=["gemv", "linear", "gemm", "gemm_ws", "linear_ws", "quant", "seq", "step"],
                     help="profile one kernel on one shape (step: the benchmark's sequence call)")
     ap.add_argument("--rows", type=int, default=13824)
     ap.add_argument("--cols", type=int, default=2560)
